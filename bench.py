@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 DSA layer: 128K-token prefill throughput and
+decode-step latency, with roofline fractions and the fp64 oracle timed on the
+host cores beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--impl reference]
+
+One step = one whole prefill of a 131072-token sequence (chunked lightning
+indexer -> per-row top-k -> sparse GQA attention) on synthetic inputs
+already resident in HBM.  Prints ONE JSON line on rank 0.  Under torchrun
+(N > 1) every rank prefills its own independent sequence (weak scaling, no
+collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "GQA-DSA prefill tok/s @128K & decode step µs; % of HBM / FP8 tensor roofline"
+UNIT = "tok/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_PER_BF16 = 2.0  # nominal dense ratio, 4.5 / 2.25 PFLOP/s
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = out.splitlines()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < len(self.FIELDS) or f[0] != str(self.gpu_index):
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# workloads
+# ----------------------------------------------------------------------------
+
+def causal_pairs(r0, n):
+    """Number of (t, s) pairs with s <= t for t in [r0, r0+n)."""
+    return n * r0 + n * (n + 1) // 2
+
+
+class PrefillBench:
+    def __init__(self, cfg, seed, device):
+        from sparse_long_context_03_b200 import dsa, inputs
+        self.dsa = dsa
+        self.cfg = cfg
+        self.d = inputs.prefill_inputs(cfg, device=device, seed=seed)
+        self.plan = dsa.PrefillPlan(cfg.L, cfg.HI, cfg.dI, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, device=device)
+        self.O = torch.empty(cfg.L, cfg.Hq, cfg.D, dtype=torch.bfloat16, device=device)
+        self.stream = torch.cuda.current_stream()
+        self.chunks = list(self.plan.chunks())
+
+    def launches_per_step(self):
+        return 2 * len(self.chunks) + 1
+
+    def step(self, ev=None):
+        """One whole prefill.  With ev (a dict of lists), brackets every
+        launch with CUDA events on the launching stream."""
+        d, p, c, dsa = self.d, self.plan, self.cfg, self.dsa
+        for r0, n in self.chunks:
+            if ev is not None:
+                a = torch.cuda.Event(enable_timing=True)
+                a.record(self.stream)
+            dsa.indexer_scores(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], r0, n, p.scores[:n])
+            if ev is not None:
+                b = torch.cuda.Event(enable_timing=True)
+                b.record(self.stream)
+            dsa.topk(p.scores[:n], r0, n, c.k, p.idx[r0:r0 + n], max_len=r0 + n, ws=p.ws)
+            if ev is not None:
+                e = torch.cuda.Event(enable_timing=True)
+                e.record(self.stream)
+                ev["indexer"].append((a, b, (r0, n)))
+                ev["topk"].append((b, e, (r0, n)))
+        if ev is not None:
+            a = torch.cuda.Event(enable_timing=True)
+            a.record(self.stream)
+        dsa.sparse_gqa_prefill(d["Q"], d["K"], d["V"], p.idx, 0, c.L, c.k, c.sm_scale, self.O)
+        if ev is not None:
+            b = torch.cuda.Event(enable_timing=True)
+            b.record(self.stream)
+            ev["attention"].append((a, b, (0, c.L)))
+
+    # algorithmic work of one launch of each kernel
+    def flops_indexer(self, r0, n):
+        c = self.cfg
+        return 2 * c.HI * c.dI * causal_pairs(r0, n)
+
+    def bytes_topk(self, r0, n):
+        return 4 * causal_pairs(r0, n) + 4 * self.cfg.k * n
+
+    def bytes_attention(self, r0, n):
+        c = self.cfg
+        t = torch.arange(r0, r0 + n, dtype=torch.float64)
+        rows = torch.clamp(t + 1, max=c.k).sum().item()
+        gather = rows * c.Hkv * 2 * c.D * 2          # each selected K and V row once per KV head
+        qo = n * c.Hq * c.D * 2 * 2                   # Q read, O written
+        return gather + qo + 4 * c.k * n              # + index rows
+
+
+def run_prefill_timed(pb, steps, warmup, world, gpu_index):
+    for _ in range(warmup):
+        pb.step()
+    torch.cuda.synchronize()
+    ev = {"indexer": [], "topk": [], "attention": []}
+    barrier(world)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_index) as clk:
+        start.record(pb.stream)
+        for _ in range(steps):
+            pb.step(ev)
+        end.record(pb.stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = start.elapsed_time(end)
+    per = {}
+    for name, lst in ev.items():
+        per[name] = [(a.elapsed_time(b), rn) for a, b, rn in lst]
+    return ms, per, clk.summary()
+
+
+def run_prefill_e2e(pb, steps, warmup):
+    """Same prefill through the public API, from pinned HOST buffers: every
+    step copies the inputs host->device, runs, and copies O back."""
+    names = ["q8", "sq", "w", "k8", "sk", "Q", "K", "V"]
+    host = {k: pb.d[k].cpu().pin_memory() for k in names}
+    dev = {k: torch.empty_like(pb.d[k]) for k in names}
+    out_host = torch.empty(pb.O.shape, dtype=pb.O.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    c, p, dsa = pb.cfg, pb.plan, pb.dsa
+
+    def one():
+        for k in names:
+            dev[k].copy_(host[k], non_blocking=True)
+        dsa.prefill_forward(p, dev["q8"], dev["sq"], dev["w"], dev["k8"], dev["sk"], dev["Q"], dev["K"], dev["V"],
+                            pb.O, c.sm_scale)
+        out_host.copy_(pb.O, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(pb.stream)
+    for _ in range(steps):
+        one()
+    e.record(pb.stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e)
+    del dev, host
+    return ms, h2d, d2h
+
+
+class DecodeBench:
+    def __init__(self, cfg, seed, device):
+        from sparse_long_context_03_b200 import dsa, inputs
+        self.dsa = dsa
+        self.cfg = cfg
+        self.d = inputs.decode_inputs(cfg, device=device, seed=seed)
+        B = self.d["q"].shape[0]
+        self.B = B
+        self.ws = torch.empty(dsa.decode_workspace_size(B, self.d["max_seq_len"], cfg.Hq, cfg.Hkv, cfg.D, cfg.k),
+                              dtype=torch.uint8, device=device)
+        self.out = torch.empty(B, cfg.Hq, cfg.D, dtype=torch.bfloat16, device=device)
+        self.stream = torch.cuda.current_stream()
+        self.lens = [int(x) for x in self.d["seq_lens"].cpu()]
+
+    def step(self):
+        d, c = self.d, self.cfg
+        self.dsa.sparse_gqa_decode(d["q"], d["q8"], d["sq"], d["w"], d["k8_cache"], d["sk_cache"], d["k_cache"],
+                                   d["v_cache"], d["block_table"], d["seq_lens"], d["max_seq_len"], c.k, c.sm_scale,
+                                   self.ws, self.out)
+
+    def algorithmic_bytes(self):
+        c = self.cfg
+        n = sum(self.lens)
+        idx_rows = sum(min(c.k, x) for x in self.lens)
+        indexer = n * (c.dI + 4)                        # FP8 key + its scale, every cached token
+        scores = n * 4 * 2                               # score row written, read by the top-k
+        gather = idx_rows * c.Hkv * 2 * c.D * 2          # selected K and V rows once per KV head
+        small = self.B * (c.Hq * c.D * 2 * 2 + c.HI * c.dI + c.HI * 4 + 4 * c.k * 2)
+        return indexer + scores + gather + small
+
+
+def run_decode_timed(db, steps, warmup):
+    for _ in range(warmup):
+        db.step()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(db.stream)
+    for _ in range(steps):
+        db.step()
+    e.record(db.stream)
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the same workload
+# ----------------------------------------------------------------------------
+
+def oracle_prefill_sample(cfg, d_host, n_rows):
+    """Oracle indexer + top-k + attention for n_rows consecutive query rows
+    centred on L/2 (their mean cost equals the whole sequence's mean row cost,
+    since a row's cost grows linearly with t).  Returns (seconds, rows, threads)."""
+    import oracle
+    L = cfg.L
+    r0 = L // 2 - n_rows // 2
+    t0 = time.perf_counter()
+    I = oracle.indexer(d_host["q8"], d_host["sq"], d_host["w"], d_host["k8"], d_host["sk"], row_begin=r0,
+                       n_rows=n_rows)
+    idx = oracle.causal_topk(I, r0, cfg.k)
+    oracle.sparse_attention(d_host["Q_rows"], d_host["K"], d_host["V"], idx, r0, cfg.sm_scale)
+    return time.perf_counter() - t0, n_rows, oracle.threads()
+
+
+def host_inputs_for_oracle(cfg, d, n_rows):
+    from sparse_long_context_03_b200 import inputs
+    L = cfg.L
+    r0 = L // 2 - n_rows // 2
+    h = {k: inputs.to_numpy_bits(d[k]) for k in ("q8", "sq", "w", "k8", "sk", "K", "V")}
+    h["Q_rows"] = inputs.to_numpy_bits(d["Q"][r0:r0 + n_rows])
+    return h
+
+
+def cpu_baseline(cfg, d, target_s=15.0):
+    import oracle
+    oracle.build()
+    h = host_inputs_for_oracle(cfg, d, 64)
+    n = max(1, oracle.threads())
+    sec, rows, thr = oracle_prefill_sample(cfg, h, n)  # calibration: one row per thread
+    # grow the sample to about target_s seconds of CPU work
+    n2 = int(max(n, min(64, rows * target_s / max(sec, 1e-3))))
+    n2 = max(n, n2 // n * n)
+    if n2 > rows:
+        h = host_inputs_for_oracle(cfg, d, n2)
+        sec, rows, thr = oracle_prefill_sample(cfg, h, n2)
+    return {"value": rows / sec, "unit": UNIT, "cores": thr, "kind": "oracle",
+            "sample": f"{rows} consecutive query rows centred on t=L/2 of the {cfg.L}-token prefill "
+                      f"(whole indexer row, top-k and attention per row, fp64), {sec:.1f} s; "
+                      f"rows/s equals tok/s because their mean cost is the sequence's mean row cost"}
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the oracle, as it stands, on the host cores
+# ----------------------------------------------------------------------------
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    from sparse_long_context_03_b200 import inputs
+    oracle.build()
+    cfg = inputs.config(args.config)
+    d = inputs.prefill_inputs(cfg, device="cpu", seed=cfg.seed)
+    n = max(1, oracle.threads())
+    h = host_inputs_for_oracle(cfg, d, n)
+    for _ in range(args.warmup):
+        oracle_prefill_sample(cfg, h, n)
+    secs = []
+    for _ in range(args.steps):
+        s, rows, thr = oracle_prefill_sample(cfg, h, n)
+        secs.append(s)
+    total = sum(secs)
+    value = args.steps * n / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: DSA prefill L={cfg.L}, Hq={cfg.Hq}, Hkv={cfg.Hkv}, D={cfg.D}, "
+                               f"HI={cfg.HI}, dI={cfg.dI}, k={cfg.k}", "seq_len": cfg.L},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
+                         "sample": f"each step: {n} consecutive query rows centred on t=L/2 (fp64 indexer row, "
+                                   f"top-k, attention)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+
+def stage_roofline(per, pb, pk, src):
+    hbm = pk["hbm_gbs"]
+    fp8 = pk["bf16_tflops"] * FP8_PER_BF16
+    out = {}
+    for name, lst in per.items():
+        if not lst:
+            continue
+        tot_ms = sum(ms for ms, _ in lst)
+        if name == "indexer":
+            work = sum(pb.flops_indexer(*rn) for _, rn in lst)
+            ach = work / (tot_ms / 1e3) / 1e12
+            out[name] = {"bound": "tensor", "achieved": ach, "peak": fp8, "unit": "TFLOP/s", "frac": ach / fp8,
+                         "ms_total": tot_ms, "launches": len(lst),
+                         "peak_note": f"FP8 = bf16 burst ({src}) x {FP8_PER_BF16} nominal ratio"}
+        else:
+            fn = pb.bytes_topk if name == "topk" else pb.bytes_attention
+            work = sum(fn(*rn) for _, rn in lst)
+            ach = work / (tot_ms / 1e3) / 1e9
+            out[name] = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                         "ms_total": tot_ms, "launches": len(lst), "peak_note": f"HBM copy ({src})"}
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=2, help="prefill workload id (see inputs.CONFIGS)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        return run_reference(args, rank, world)
+
+    rank, world, local = dist_setup(args.gpus)
+    from sparse_long_context_03_b200 import build, inputs
+    if rank == 0:
+        build.build()
+    barrier(world)
+
+    pk, src = peaks()
+    cfg = inputs.config(args.config)
+    pb = PrefillBench(cfg, seed=cfg.seed + 7919 * rank, device="cuda")
+    chunk_rows = pb.plan.chunk_rows
+    ms, per, clocks = run_prefill_timed(pb, args.steps, args.warmup, world, local)
+    ms_max = max_over_ranks(ms, world)
+    value = world * cfg.L * args.steps / (ms_max / 1e3)
+    stages = stage_roofline(per, pb, pk, src)
+    dominant = max(stages, key=lambda k: stages[k]["ms_total"])
+    dom = dict(stages[dominant])
+    dom_line = {"kernel": dominant, "bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"],
+                "unit": dom["unit"], "frac": dom["frac"], "traffic": None, "peak_source": dom["peak_note"]}
+
+    e2e = None
+    if not args.no_e2e:
+        ems, h2d, d2h = run_prefill_e2e(pb, max(1, min(args.steps, 3)), 1)
+        n_e2e = max(1, min(args.steps, 3))
+        ems = max_over_ranks(ems, world)
+        e2e = {"value": world * cfg.L * n_e2e / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems / n_e2e}
+
+    decode = None
+    if not args.no_decode:
+        del pb
+        torch.cuda.empty_cache()
+        dcfg = inputs.config(3)
+        db = DecodeBench(dcfg, seed=dcfg.seed + 7919 * rank, device="cuda")
+        us = 1e3 * max_over_ranks(run_decode_timed(db, max(args.steps, 20), max(args.warmup, 3)), world)
+        byts = db.algorithmic_bytes()
+        decode = {"workload": f"{dcfg.name}: B={db.B}, cached lengths U[{dcfg.len_lo},{dcfg.len_hi}] "
+                              f"(mean {statistics.mean(db.lens):.0f}), page 64, k={dcfg.k}",
+                  "step_us": us, "higher_is_better": False,
+                  "roofline": {"bound": "hbm", "achieved": byts / (us / 1e6) / 1e9, "peak": pk["hbm_gbs"],
+                               "unit": "GB/s", "frac": byts / (us / 1e6) / 1e9 / pk["hbm_gbs"],
+                               "algorithmic_bytes": byts},
+                  "gpu_launches_per_step": 4}
+        pb = None
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        d_cpu = inputs.prefill_inputs(cfg, device="cuda", seed=cfg.seed)
+        cpu = cpu_baseline(cfg, d_cpu)
+        del d_cpu
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp8-e4m3 indexer / bf16 attention (fp32 accumulate)",
+            "data": "synthetic (seeded; shapes and distributions of the 128K prefill workload)",
+            "config": {"workload": f"{cfg.name}: DSA prefill L={cfg.L}, batch 1 per GPU, Hq={cfg.Hq}, Hkv={cfg.Hkv}, "
+                                   f"D={cfg.D}, HI={cfg.HI}, dI={cfg.dI}, k={cfg.k}, query chunks of {chunk_rows} rows",
+                       "global_batch": world, "seq_len": cfg.L, "parallelism": f"independent sequences x{world}",
+                       "l2": "inputs larger than L2 (4 GiB score chunks, 1 GiB Q) between launches"},
+            "roofline": dom_line, "stages": stages, "clocks": clocks, "gpu_launches": None,
+            "e2e": e2e, "decode": decode, "cpu_baseline": cpu,
+        }
+        line["gpu_launches"] = sum(len(v) for v in per.values())
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,202 @@
+/*
+ * dsa.h -- C ABI of libdsa.so, the B200 (sm_100a) GQA-adapted DeepSeek Sparse
+ * Attention (DSA) layer: lightning indexer -> causal top-k -> sparse GQA
+ * attention, for prefill and for decode over a paged KV cache.
+ *
+ * Sources (web pages on the Kwai Keye-VL-2.0 technical report):
+ *   [REVIEW]  "Kwai Keye-VL-2.0 Technical Report" paper review
+ *             (xllm-io.github.io), section 三 "技术架构", "核心公式".
+ *   [REPORT]  "快手开源 Kwai Keye-VL-2.0-30B-A3B：面向长视频理解与智能体智能的
+ *             MoE 多模态模型" (translation of the report), sections 2.3.1,
+ *             2.3.2, 5.1.2, 5.2.1 and 5.3.
+ *
+ * Conventions for every call
+ * --------------------------
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller.  Layouts are
+ *    row-major and dense unless a leading dimension is passed.  Shapes below
+ *    use [a, b, c] with c fastest.
+ *  - The library never allocates, frees or synchronises.  Temporary memory
+ *    comes from a caller-provided workspace whose size a *_workspace_size()
+ *    query returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and keep no state between calls, so separate calls on separate
+ *    streams with separate buffers may run concurrently.
+ *  - Arguments are validated on the host before any CUDA call.  On an error
+ *    nothing is launched and no output is touched.  DSA_ERR_CUDA means a
+ *    launch failed; the CUDA error string is available from
+ *    dsa_last_error_string() on the calling thread.
+ *  - FP8 means OCP e4m3fn bytes; the real value of a stored byte is
+ *    e4m3(byte) * scale, one float scale per token.  bf16 tensors are passed
+ *    as uint16_t bit patterns.  NaN / Inf inputs give unspecified results.
+ *  - Index tensors are int32.  Selected-index rows are ascending and padded
+ *    with -1.  Entries of an index row that fall outside the causally visible
+ *    range are skipped by the attention kernels, so a corrupt row cannot make
+ *    them read out of bounds.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#define DSA_VERSION 100      /* 1.0.0 */
+#define DSA_PAGE_SIZE 64     /* tokens per KV-cache page */
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad range */
+    DSA_ERR_UNSUPPORTED_SHAPE = 2, /* a head count or head dim this build has no kernel for */
+    DSA_ERR_WORKSPACE = 3,         /* workspace missing or smaller than the size query */
+    DSA_ERR_CUDA = 4,              /* a kernel launch failed */
+    DSA_ERR_TIMEOUT = 5            /* reserved: a bounded device-side wait gave up */
+} dsa_status_t;
+
+/* Human-readable name of a status code (static storage). */
+DSA_API const char *dsa_status_string(dsa_status_t s);
+/* DSA_VERSION of the loaded library. */
+DSA_API int dsa_version(void);
+/* Text of the last CUDA error seen by a dsa_* call on this thread ("" if none). */
+DSA_API const char *dsa_last_error_string(void);
+
+/* ------------------------------------------------------------------------
+ * Lightning-indexer scores (prefill), one chunk of query rows.
+ *
+ * [REVIEW] 核心公式, indexer score; [REPORT] 2.3.1 (one key head shared by all
+ * indexer heads, FP8, ReLU scoring):
+ *     I[t,s] = sum_{j<HI} w[t,j] * ReLU( qI[t,j] . kI[s] ),   0 <= s <= t,
+ *     qI[t,j,c] = e4m3(q8[t,j,c]) * q_scale[t],  kI[s,c] = e4m3(k8[s,c]) * k_scale[s].
+ * The score matrix is produced one chunk of query rows at a time ([REPORT]
+ * 5.2.1: the chunked indexer bounds peak memory).
+ *
+ *   q8       [L, HI, dI] e4m3      q_scale [L] float     w [L, HI] float
+ *   k8       [L, dI]     e4m3      k_scale [L] float
+ *   rows     t in [row_begin, row_begin + n_rows), 0 <= row_begin, row_begin + n_rows <= L
+ *   scores   [n_rows, ld_scores] float; row r holds query t = row_begin + r;
+ *            columns 0..t are written, columns > t are left unspecified.
+ *            ld_scores >= row_begin + n_rows and ld_scores % 4 == 0.
+ * Supported: dI in {32, 64, 128}; HI in {4, 8, 16, 32, 64}.
+ * All scale factors must be positive (they commute with the ReLU).
+ * ------------------------------------------------------------------------ */
+DSA_API dsa_status_t dsa_indexer_scores(const uint8_t *q8, const float *q_scale, const float *w,
+                                const uint8_t *k8, const float *k_scale,
+                                int L, int HI, int dI, int row_begin, int n_rows,
+                                float *scores, int64_t ld_scores, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Per-row top-k selection.
+ *
+ * [REVIEW] 核心公式, Omega_t = { s | I[t,s] in Top-k(I[t,:]) }; [REPORT] 2.3.1;
+ * [REPORT] 5.1.2 (a row with fewer than k visible entries keeps all of them);
+ * [REPORT] 5.2.1 (the selection must be deterministic).
+ * Row r has n_r candidates scores[r * ld_scores + 0 .. n_r-1]:
+ *   row_len == NULL: n_r = row_begin + r + 1 (causal prefill rows),
+ *   row_len != NULL: n_r = row_len[r] (device int32 [n_rows]), clamped to [0, max_len].
+ * Output idx [n_rows, k]: if n_r <= k, the indices 0..n_r-1; otherwise the k
+ * indices of the largest scores, ties broken toward the lower index, -0.0 and
+ * +0.0 equal.  Indices ascending, padded with -1.
+ *   max_len  upper bound of every n_r (the host sizes grids with it);
+ *            ld_scores >= max_len and ld_scores % 4 == 0.
+ *   ws       device workspace of at least dsa_topk_workspace_size() bytes
+ *            (may be NULL when that size is 0).
+ * ------------------------------------------------------------------------ */
+DSA_API size_t dsa_topk_workspace_size(int n_rows, int max_len, int k);
+DSA_API dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, int row_begin, int n_rows,
+                      const int32_t *row_len, int max_len, int k, int32_t *idx,
+                      void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Sparse GQA attention (prefill), one chunk of query rows.
+ *
+ * [REVIEW] 核心公式, u[t,g] = Attn(h[t,g], { c[s,g] | s in Omega_t });
+ * [REPORT] 2.3.2: one index set Omega_t serves every KV group g; the group
+ * outputs are concatenated.  Head h reads group g = h / (Hq / Hkv):
+ *     O[t,h] = sum_{s in Omega_t} softmax_s( sm_scale * Q[t,h] . K[s,g] ) V[s,g]
+ *     lse[t,h] = log sum_{s in Omega_t} exp( sm_scale * Q[t,h] . K[s,g] )
+ * Only the first min(k, t+1) entries of an index row are visited ([REPORT]
+ * 5.1.2); entries outside [0, t] are skipped.
+ *
+ *   Q    [n_rows, Hq, D] bf16 (row r is query t = row_begin + r)
+ *   K, V [>= row_begin + n_rows, Hkv, D] bf16
+ *   idx  [n_rows, k] int32 (from dsa_topk)
+ *   O    [n_rows, Hq, D] bf16;  lse [n_rows, Hq] float, may be NULL.
+ * Supported: D in {64, 128}; Hq % Hkv == 0 with Hq / Hkv <= 8.
+ * A row with no valid index writes O = 0 and lse = -inf.
+ * ------------------------------------------------------------------------ */
+DSA_API dsa_status_t dsa_sparse_gqa_prefill(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                                    const int32_t *idx, int row_begin, int n_rows,
+                                    int Hq, int Hkv, int D, int k, float sm_scale,
+                                    uint16_t *O, float *lse, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Decode over a paged cache: one new query token per sequence.
+ *
+ * [REPORT] 5.3 (DSA decode); formulas as above with t = seq_lens[b] - 1: the
+ * new token's K, V and indexer key are already in the cache.  Logical token s
+ * of sequence b lives in page block_table[b * max_pages + s / 64], slot s % 64.
+ *
+ *   q             [B, Hq, D] bf16          q8 [B, HI, dI] e4m3
+ *   q_scale       [B] float                w  [B, HI] float
+ *   k8_cache      [num_pages, 64, dI] e4m3 k_scale_cache [num_pages, 64] float
+ *   k_cache,
+ *   v_cache       [num_pages, 64, Hkv, D] bf16
+ *   block_table   [B, max_pages] int32 (entries past a sequence's end unused)
+ *   seq_lens      [B] int32, 1 <= seq_lens[b] <= min(max_seq_len, 64 * max_pages)
+ *   max_seq_len   host-side upper bound of seq_lens (sizes grids and workspace)
+ *   out           [B, Hq, D] bf16
+ *   idx_out       [B, k] int32 selected indices, may be NULL
+ *   ws            >= dsa_decode_workspace_size(...) bytes
+ * A token on a page id outside [0, num_pages) scores -inf and is skipped by
+ * the attention.
+ * dsa_sparse_gqa_decode runs the three stages below on `stream`:
+ * scores (dsa_decode_indexer_scores) -> top-k (dsa_topk with row_len =
+ * seq_lens) -> attention (dsa_sparse_gqa_decode_attention).
+ * ------------------------------------------------------------------------ */
+DSA_API size_t dsa_decode_workspace_size(int B, int max_seq_len, int Hq, int Hkv, int D, int k);
+DSA_API dsa_status_t dsa_sparse_gqa_decode(const uint16_t *q, const uint8_t *q8, const float *q_scale,
+                                   const float *w,
+                                   const uint8_t *k8_cache, const float *k_scale_cache,
+                                   const uint16_t *k_cache, const uint16_t *v_cache,
+                                   const int32_t *block_table, int max_pages, int num_pages,
+                                   const int32_t *seq_lens, int max_seq_len,
+                                   int B, int Hq, int Hkv, int D, int HI, int dI, int k,
+                                   float sm_scale, void *ws, size_t ws_bytes,
+                                   uint16_t *out, int32_t *idx_out, void *stream);
+
+/* Decode stage 1: indexer scores of each sequence's query against its cached
+ * keys.  scores [B, ld_scores] float, columns 0..seq_lens[b]-1 written;
+ * ld_scores >= max_seq_len and ld_scores % 4 == 0.  Same formula and shape
+ * support as dsa_indexer_scores. */
+DSA_API dsa_status_t dsa_decode_indexer_scores(const uint8_t *q8, const float *q_scale, const float *w,
+                                       const uint8_t *k8_cache, const float *k_scale_cache,
+                                       const int32_t *block_table, int max_pages, int num_pages,
+                                       const int32_t *seq_lens, int max_seq_len,
+                                       int B, int HI, int dI,
+                                       float *scores, int64_t ld_scores, void *stream);
+
+/* Decode stage 3: attention of each sequence's query over the selected rows
+ * idx [B, k] (entries outside [0, seq_lens[b]) skipped), read through the
+ * block table.  lse [B, Hq] may be NULL.  ws >=
+ * dsa_decode_attention_workspace_size(B, Hq, Hkv, D, k) bytes. */
+DSA_API size_t dsa_decode_attention_workspace_size(int B, int Hq, int Hkv, int D, int k);
+DSA_API dsa_status_t dsa_sparse_gqa_decode_attention(const uint16_t *q,
+                                             const uint16_t *k_cache, const uint16_t *v_cache,
+                                             const int32_t *block_table, int max_pages, int num_pages,
+                                             const int32_t *seq_lens, const int32_t *idx,
+                                             int B, int Hq, int Hkv, int D, int k, float sm_scale,
+                                             void *ws, size_t ws_bytes,
+                                             uint16_t *out, float *lse, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSA_H_ */

@@ -1,0 +1,184 @@
+// abi.cu -- the extern "C" entry points declared in include/dsa.h.
+//
+// Host code here only validates arguments, sizes workspaces and launches the
+// kernels on the caller's stream.  It never allocates, frees or synchronises.
+// Validation comes before any CUDA call, so an invalid call touches nothing.
+#include <cstring>
+
+#include "dsa.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+dsa_status_t cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return DSA_OK;
+    std::strncpy(g_last_error, cudaGetErrorString(e), sizeof(g_last_error) - 1);
+    g_last_error[sizeof(g_last_error) - 1] = '\0';
+    return DSA_ERR_CUDA;
+}
+
+inline cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Layout of the decode workspace: [scores B x ld][idx B x k][attention partials].
+struct DecodeWs {
+    int64_t ld;
+    size_t scores_off, idx_off, topk_off, attn_off, total;
+};
+
+DecodeWs decode_ws_layout(int B, int max_seq_len, int Hq, int Hkv, int D, int k) {
+    DecodeWs w{};
+    w.ld = (int64_t)align_up((size_t)(max_seq_len > 0 ? max_seq_len : 1), 4);
+    w.scores_off = 0;
+    w.idx_off = align_up(w.scores_off + (size_t)B * w.ld * sizeof(float), 256);
+    w.topk_off = align_up(w.idx_off + (size_t)B * k * sizeof(int32_t), 256);
+    w.attn_off = align_up(w.topk_off + dsa::topk_workspace_bytes(B, max_seq_len, k), 256);
+    w.total = align_up(w.attn_off + dsa::decode_attention_workspace_bytes(B, Hq, Hkv, D, k), 256);
+    return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *dsa_status_string(dsa_status_t s) {
+    switch (s) {
+        case DSA_OK: return "DSA_OK";
+        case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG";
+        case DSA_ERR_UNSUPPORTED_SHAPE: return "DSA_ERR_UNSUPPORTED_SHAPE";
+        case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+        case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+        case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT";
+    }
+    return "DSA_ERR_UNKNOWN";
+}
+
+int dsa_version(void) { return DSA_VERSION; }
+
+const char *dsa_last_error_string(void) { return g_last_error; }
+
+dsa_status_t dsa_indexer_scores(const uint8_t *q8, const float *q_scale, const float *w, const uint8_t *k8,
+                                const float *k_scale, int L, int HI, int dI, int row_begin, int n_rows,
+                                float *scores, int64_t ld_scores, void *stream) {
+    if (L < 1 || row_begin < 0 || n_rows < 0 || (int64_t)row_begin + n_rows > L) return DSA_ERR_INVALID_ARG;
+    if (!dsa::indexer_shape_supported(HI, dI)) return DSA_ERR_UNSUPPORTED_SHAPE;
+    if (n_rows == 0) return DSA_OK;
+    if (!q8 || !q_scale || !w || !k8 || !k_scale || !scores) return DSA_ERR_INVALID_ARG;
+    if (ld_scores < (int64_t)row_begin + n_rows || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
+    return cuda_status(dsa::launch_indexer_prefill_mma(q8, q_scale, w, k8, k_scale, HI, dI, row_begin, n_rows,
+                                                       scores, ld_scores, as_stream(stream)));
+}
+
+size_t dsa_topk_workspace_size(int n_rows, int max_len, int k) {
+    if (n_rows < 0 || max_len < 0 || k < 1) return 0;
+    return dsa::topk_workspace_bytes(n_rows, max_len, k);
+}
+
+dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, int row_begin, int n_rows, const int32_t *row_len,
+                      int max_len, int k, int32_t *idx, void *ws, size_t ws_bytes, void *stream) {
+    if (n_rows < 0 || row_begin < 0 || k < 1 || max_len < 0) return DSA_ERR_INVALID_ARG;
+    if (row_len == nullptr && (int64_t)row_begin + n_rows > max_len) return DSA_ERR_INVALID_ARG;
+    if (n_rows == 0) return DSA_OK;
+    if (!scores || !idx) return DSA_ERR_INVALID_ARG;
+    if (ld_scores < max_len || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
+    const size_t need = dsa::topk_workspace_bytes(n_rows, max_len, k);
+    if (ws_bytes < need || (need > 0 && ws == nullptr)) return DSA_ERR_WORKSPACE;
+    return cuda_status(dsa::launch_topk(scores, ld_scores, row_begin, n_rows, row_len, max_len, k, idx, ws,
+                                        ws_bytes, as_stream(stream)));
+}
+
+dsa_status_t dsa_sparse_gqa_prefill(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const int32_t *idx,
+                                    int row_begin, int n_rows, int Hq, int Hkv, int D, int k, float sm_scale,
+                                    uint16_t *O, float *lse, void *stream) {
+    if (row_begin < 0 || n_rows < 0 || k < 1 || Hq < 1 || Hkv < 1) return DSA_ERR_INVALID_ARG;
+    if (!dsa::attention_shape_supported(Hq, Hkv, D)) return DSA_ERR_UNSUPPORTED_SHAPE;
+    if (n_rows == 0) return DSA_OK;
+    if (!Q || !K || !V || !idx || !O) return DSA_ERR_INVALID_ARG;
+    return cuda_status(dsa::launch_sparse_prefill(Q, K, V, idx, row_begin, n_rows, Hq, Hkv, D, k, sm_scale, O, lse,
+                                                  as_stream(stream)));
+}
+
+static dsa_status_t check_decode_common(const int32_t *block_table, int max_pages, int num_pages,
+                                        const int32_t *seq_lens, int max_seq_len, int B) {
+    if (B < 0 || max_pages < 1 || num_pages < 1 || max_seq_len < 0) return DSA_ERR_INVALID_ARG;
+    if ((int64_t)max_seq_len > (int64_t)max_pages * DSA_PAGE_SIZE) return DSA_ERR_INVALID_ARG;
+    if (B > 0 && (!block_table || !seq_lens)) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+}
+
+dsa_status_t dsa_decode_indexer_scores(const uint8_t *q8, const float *q_scale, const float *w,
+                                       const uint8_t *k8_cache, const float *k_scale_cache,
+                                       const int32_t *block_table, int max_pages, int num_pages,
+                                       const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI,
+                                       float *scores, int64_t ld_scores, void *stream) {
+    dsa_status_t st = check_decode_common(block_table, max_pages, num_pages, seq_lens, max_seq_len, B);
+    if (st != DSA_OK) return st;
+    if (!dsa::indexer_shape_supported(HI, dI)) return DSA_ERR_UNSUPPORTED_SHAPE;
+    if (B == 0 || max_seq_len == 0) return DSA_OK;
+    if (!q8 || !q_scale || !w || !k8_cache || !k_scale_cache || !scores) return DSA_ERR_INVALID_ARG;
+    if (ld_scores < max_seq_len || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
+    return cuda_status(dsa::launch_indexer_decode(q8, q_scale, w, k8_cache, k_scale_cache, block_table, max_pages,
+                                                  num_pages, seq_lens, max_seq_len, B, HI, dI, scores, ld_scores,
+                                                  as_stream(stream)));
+}
+
+size_t dsa_decode_attention_workspace_size(int B, int Hq, int Hkv, int D, int k) {
+    if (B < 0 || Hkv < 1 || k < 1 || D < 1) return 0;
+    return dsa::decode_attention_workspace_bytes(B, Hq, Hkv, D, k);
+}
+
+dsa_status_t dsa_sparse_gqa_decode_attention(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                                             const int32_t *block_table, int max_pages, int num_pages,
+                                             const int32_t *seq_lens, const int32_t *idx, int B, int Hq, int Hkv,
+                                             int D, int k, float sm_scale, void *ws, size_t ws_bytes,
+                                             uint16_t *out, float *lse, void *stream) {
+    if (B < 0 || k < 1 || Hq < 1 || Hkv < 1 || max_pages < 1 || num_pages < 1) return DSA_ERR_INVALID_ARG;
+    if (!dsa::attention_shape_supported(Hq, Hkv, D)) return DSA_ERR_UNSUPPORTED_SHAPE;
+    if (B == 0) return DSA_OK;
+    if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !idx || !out) return DSA_ERR_INVALID_ARG;
+    if (ws == nullptr || ws_bytes < dsa::decode_attention_workspace_bytes(B, Hq, Hkv, D, k)) return DSA_ERR_WORKSPACE;
+    return cuda_status(dsa::launch_sparse_decode(q, k_cache, v_cache, block_table, max_pages, num_pages, seq_lens,
+                                                 idx, B, Hq, Hkv, D, k, sm_scale, ws, ws_bytes, out, lse,
+                                                 as_stream(stream)));
+}
+
+size_t dsa_decode_workspace_size(int B, int max_seq_len, int Hq, int Hkv, int D, int k) {
+    if (B < 0 || max_seq_len < 0 || Hkv < 1 || k < 1 || D < 1) return 0;
+    return decode_ws_layout(B, max_seq_len, Hq, Hkv, D, k).total;
+}
+
+dsa_status_t dsa_sparse_gqa_decode(const uint16_t *q, const uint8_t *q8, const float *q_scale, const float *w,
+                                   const uint8_t *k8_cache, const float *k_scale_cache, const uint16_t *k_cache,
+                                   const uint16_t *v_cache, const int32_t *block_table, int max_pages,
+                                   int num_pages, const int32_t *seq_lens, int max_seq_len, int B, int Hq, int Hkv,
+                                   int D, int HI, int dI, int k, float sm_scale, void *ws, size_t ws_bytes,
+                                   uint16_t *out, int32_t *idx_out, void *stream) {
+    dsa_status_t st = check_decode_common(block_table, max_pages, num_pages, seq_lens, max_seq_len, B);
+    if (st != DSA_OK) return st;
+    if (k < 1 || Hq < 1 || Hkv < 1) return DSA_ERR_INVALID_ARG;
+    if (!dsa::indexer_shape_supported(HI, dI) || !dsa::attention_shape_supported(Hq, Hkv, D))
+        return DSA_ERR_UNSUPPORTED_SHAPE;
+    if (B == 0) return DSA_OK;
+    if (!q || !q8 || !q_scale || !w || !k8_cache || !k_scale_cache || !k_cache || !v_cache || !out)
+        return DSA_ERR_INVALID_ARG;
+    const DecodeWs L = decode_ws_layout(B, max_seq_len, Hq, Hkv, D, k);
+    if (ws == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+    char *base = static_cast<char *>(ws);
+    float *scores = reinterpret_cast<float *>(base + L.scores_off);
+    int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(base + L.idx_off);
+    cudaStream_t s = as_stream(stream);
+    cudaError_t e = dsa::launch_indexer_decode(q8, q_scale, w, k8_cache, k_scale_cache, block_table, max_pages,
+                                               num_pages, seq_lens, max_seq_len, B, HI, dI, scores, L.ld, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = dsa::launch_topk(scores, L.ld, 0, B, seq_lens, max_seq_len, k, idx, base + L.topk_off,
+                         dsa::topk_workspace_bytes(B, max_seq_len, k), s);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = dsa::launch_sparse_decode(q, k_cache, v_cache, block_table, max_pages, num_pages, seq_lens, idx, B, Hq, Hkv,
+                                  D, k, sm_scale, base + L.attn_off, L.total - L.attn_off, out, nullptr, s);
+    return cuda_status(e);
+}
+
+}  // extern "C"

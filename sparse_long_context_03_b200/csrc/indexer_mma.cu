@@ -1,0 +1,253 @@
+// indexer_mma.cu -- lightning-indexer scores on warp-level FP8 tensor-core MMA.
+//
+// "Kwai Keye-VL-2.0 Technical Report" review (xllm-io), 核心公式, indexer:
+//     I[t,s] = sum_j w[t,j] * ReLU(qI[t,j] . kI[s])
+// with one key head shared by every indexer head and FP8 inputs (report
+// translation, section 2.3.1).  The per-token scales are positive, so
+//     I[t,s] = sq[t] * sk[s] * sum_j w[t,j] * ReLU(q8[t,j] . k8[s])
+// where the byte dot products run on the tensor cores (e4m3 x e4m3 -> fp32).
+//
+// GEMM orientation: M = keys (16 per warp), N = indexer heads (8 per MMA
+// tile), K = dI.  Each thread's accumulators cover two keys and two heads per
+// tile, so the ReLU, the weighted head sum and the causal mask are applied in
+// registers; the head sum finishes with two xor-shuffles across the 4 lanes
+// that share a key.
+//
+// Two kernels share this: the paged decode indexer (one query per sequence,
+// keys read through the block table) and a prefill fallback used for shapes
+// the tcgen05 kernel does not take.
+#include <type_traits>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dsa {
+
+namespace {
+
+// Score contribution of one query against the warp's 16 keys.  a: key
+// fragments [KS][4]; b(nt, ks, half) yields the query fragment; wv(nt, i) the
+// head weights.  Returns the two per-key sums (keys gid and gid+8), complete
+// on every lane after the shuffles.
+template <int KS, int NT, typename BF, typename WF>
+__device__ __forceinline__ void score_16keys(const uint32_t (&a)[KS][4], BF bfrag, WF wv, float &p0, float &p1) {
+    p0 = 0.f;
+    p1 = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) mma_e4m3_16832(acc, a[ks], bfrag(nt, ks, 0), bfrag(nt, ks, 1));
+        const float wa = wv(nt, 0), wb = wv(nt, 1);
+        p0 = fmaf(wa, fmaxf(acc[0], 0.f), p0);
+        p0 = fmaf(wb, fmaxf(acc[1], 0.f), p0);
+        p1 = fmaf(wa, fmaxf(acc[2], 0.f), p1);
+        p1 = fmaf(wb, fmaxf(acc[3], 0.f), p1);
+    }
+    p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
+    p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
+    p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
+    p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
+}
+
+// Key fragments of 16 consecutive key rows (row stride DI bytes) for the
+// m16n8k32 A operand: a[ks][0] row gid, bytes ks*32 + tig*4; [1] row gid+8;
+// [2] row gid, bytes +16; [3] row gid+8, bytes +16.
+template <int DI>
+__device__ __forceinline__ void load_key_frags(uint32_t (&a)[DI / 32][4], const uint8_t *row0, const uint8_t *row8,
+                                               bool ok0, bool ok8, int tig) {
+#pragma unroll
+    for (int ks = 0; ks < DI / 32; ++ks) {
+        const int off = ks * 32 + tig * 4;
+        a[ks][0] = ok0 ? __ldg(reinterpret_cast<const uint32_t *>(row0 + off)) : 0u;
+        a[ks][1] = ok8 ? __ldg(reinterpret_cast<const uint32_t *>(row8 + off)) : 0u;
+        a[ks][2] = ok0 ? __ldg(reinterpret_cast<const uint32_t *>(row0 + off + 16)) : 0u;
+        a[ks][3] = ok8 ? __ldg(reinterpret_cast<const uint32_t *>(row8 + off + 16)) : 0u;
+    }
+}
+
+constexpr int kKeysPerCta = 128;  // 8 warps x 16 keys
+
+// Queries per prefill CTA: as many as fit 40 KB of static shared memory.
+template <int DI, int NT>
+constexpr int prefill_qb() {
+    constexpr int per_query = NT * 8 * (DI + 16);
+    return per_query * 16 <= 40960 ? 16 : (per_query * 8 <= 40960 ? 8 : 4);
+}
+
+template <int DI, int NT>
+__global__ void __launch_bounds__(256) indexer_prefill_mma_kernel(
+    const uint8_t *__restrict__ q8, const float *__restrict__ sq, const float *__restrict__ w,
+    const uint8_t *__restrict__ k8, const float *__restrict__ sk, int HI, int row_begin, int n_rows,
+    float *__restrict__ scores, int64_t ld) {
+    constexpr int KS = DI / 32;
+    constexpr int HP = NT * 8;      // heads padded to the MMA tile
+    constexpr int QROW = DI + 16;   // padded smem row: conflict-free fragment loads
+    constexpr int kPrefillQB = prefill_qb<DI, NT>();
+    __shared__ __align__(16) uint8_t q_s[kPrefillQB * HP * QROW];
+    __shared__ float w_s[kPrefillQB][HP];
+    __shared__ float sq_s[kPrefillQB];
+
+    const int t0 = row_begin + blockIdx.y * kPrefillQB;
+    const int t_last = min(t0 + kPrefillQB, row_begin + n_rows) - 1;
+    const int s0 = blockIdx.x * kKeysPerCta;
+    if (s0 > t_last) return;  // tile entirely above the causal diagonal
+
+    for (int i = threadIdx.x; i < kPrefillQB * HP * (DI / 16); i += blockDim.x) {
+        const int row = i / (DI / 16), c16 = i % (DI / 16);
+        const int qi = row / HP, h = row % HP, t = t0 + qi;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (t <= t_last && h < HI) v = __ldg(reinterpret_cast<const uint4 *>(q8 + ((size_t)t * HI + h) * DI) + c16);
+        *reinterpret_cast<uint4 *>(q_s + row * QROW + c16 * 16) = v;
+    }
+    for (int i = threadIdx.x; i < kPrefillQB * HP; i += blockDim.x) {
+        const int qi = i / HP, h = i % HP, t = t0 + qi;
+        w_s[qi][h] = (t <= t_last && h < HI) ? __ldg(w + (size_t)t * HI + h) : 0.f;
+    }
+    if (threadIdx.x < kPrefillQB) {
+        const int t = t0 + threadIdx.x;
+        sq_s[threadIdx.x] = t <= t_last ? __ldg(sq + t) : 0.f;
+    }
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = lane_id(), gid = lane >> 2, tig = lane & 3;
+    const int sb = s0 + warp * 16;
+    if (sb > t_last) return;
+    const int key0 = sb + gid, key8 = key0 + 8;
+    uint32_t a[KS][4];
+    load_key_frags<DI>(a, k8 + (size_t)key0 * DI, k8 + (size_t)key8 * DI, key0 <= t_last, key8 <= t_last, tig);
+    const float sk0 = key0 <= t_last ? __ldg(sk + key0) : 0.f;
+    const float sk8 = key8 <= t_last ? __ldg(sk + key8) : 0.f;
+
+    for (int qi = 0; qi < kPrefillQB; ++qi) {
+        const int t = t0 + qi;
+        if (t > t_last) break;
+        if (sb > t) continue;
+        const uint8_t *qrow = q_s + (qi * HP) * QROW;
+        float p0, p1;
+        score_16keys<KS, NT>(
+            a,
+            [&](int nt, int ks, int half) {
+                return *reinterpret_cast<const uint32_t *>(qrow + (nt * 8 + gid) * QROW + ks * 32 + tig * 4 + half * 16);
+            },
+            [&](int nt, int i) { return w_s[qi][nt * 8 + tig * 2 + i]; }, p0, p1);
+        const float f = sq_s[qi];
+        float *srow = scores + (size_t)(t - row_begin) * ld;
+        if (tig == 0 && key0 <= t) srow[key0] = p0 * f * sk0;
+        if (tig == 1 && key8 <= t) srow[key8] = p1 * f * sk8;
+    }
+}
+
+template <int DI, int NT>
+__global__ void __launch_bounds__(256) indexer_decode_mma_kernel(
+    const uint8_t *__restrict__ q8, const float *__restrict__ sq, const float *__restrict__ w,
+    const uint8_t *__restrict__ k8c, const float *__restrict__ skc, const int32_t *__restrict__ block_table,
+    int max_pages, int num_pages, const int32_t *__restrict__ seq_lens, int max_seq_len, int HI,
+    float *__restrict__ scores, int64_t ld) {
+    constexpr int KS = DI / 32;
+    const int b = blockIdx.y;
+    const int n = min(min(__ldg(seq_lens + b), max_seq_len), max_pages * kPage);
+    const int warp = threadIdx.x >> 5, lane = lane_id(), gid = lane >> 2, tig = lane & 3;
+    const int sb = blockIdx.x * kKeysPerCta + warp * 16;
+    if (sb >= n) return;
+
+    // Query fragments (m16n8k32 B operand, column n = head): b0 bytes
+    // ks*32 + tig*4 of head nt*8+gid, b1 the same +16.
+    uint32_t qf[NT][KS][2];
+    float wf[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int h = nt * 8 + gid;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            const uint8_t *qp = q8 + ((size_t)b * HI + h) * DI + ks * 32 + tig * 4;
+            qf[nt][ks][0] = h < HI ? __ldg(reinterpret_cast<const uint32_t *>(qp)) : 0u;
+            qf[nt][ks][1] = h < HI ? __ldg(reinterpret_cast<const uint32_t *>(qp + 16)) : 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int hw = nt * 8 + tig * 2 + i;
+            wf[nt][i] = hw < HI ? __ldg(w + (size_t)b * HI + hw) : 0.f;
+        }
+    }
+
+    const int page = __ldg(block_table + (size_t)b * max_pages + sb / kPage);
+    const bool page_ok = page >= 0 && page < num_pages;
+    const int key0 = sb + gid, key8 = key0 + 8;
+    const size_t slot0 = (size_t)(page_ok ? page : 0) * kPage + (key0 % kPage);
+    const size_t slot8 = slot0 + 8;
+    uint32_t a[KS][4];
+    load_key_frags<DI>(a, k8c + slot0 * DI, k8c + slot8 * DI, page_ok && key0 < n, page_ok && key8 < n, tig);
+    const float sk0 = (page_ok && key0 < n) ? __ldg(skc + slot0) : 0.f;
+    const float sk8 = (page_ok && key8 < n) ? __ldg(skc + slot8) : 0.f;
+
+    float p0, p1;
+    score_16keys<KS, NT>(
+        a, [&](int nt, int ks, int half) { return qf[nt][ks][half]; }, [&](int nt, int i) { return wf[nt][i]; }, p0,
+        p1);
+    const float f = __ldg(sq + b);
+    float *srow = scores + (size_t)b * ld;
+    if (tig == 0 && key0 < n) srow[key0] = page_ok ? p0 * f * sk0 : -INFINITY;
+    if (tig == 1 && key8 < n) srow[key8] = page_ok ? p1 * f * sk8 : -INFINITY;
+}
+
+// Calls launch(integral_constant<DI>, integral_constant<NT>) for a supported
+// (HI, dI); HI = 4 uses one 8-wide head tile with the upper half zeroed.
+template <typename F>
+bool dispatch_shape(int HI, int dI, F &&launch) {
+    auto by_nt = [&](auto di) -> bool {
+        switch (HI) {
+            case 4:
+            case 8: return launch(di, std::integral_constant<int, 1>{});
+            case 16: return launch(di, std::integral_constant<int, 2>{});
+            case 32: return launch(di, std::integral_constant<int, 4>{});
+            case 64: return launch(di, std::integral_constant<int, 8>{});
+            default: return false;
+        }
+    };
+    switch (dI) {
+        case 32: return by_nt(std::integral_constant<int, 32>{});
+        case 64: return by_nt(std::integral_constant<int, 64>{});
+        case 128: return by_nt(std::integral_constant<int, 128>{});
+        default: return false;
+    }
+}
+
+}  // namespace
+
+bool indexer_shape_supported(int HI, int dI) {
+    return (HI == 4 || HI == 8 || HI == 16 || HI == 32 || HI == 64) && (dI == 32 || dI == 64 || dI == 128);
+}
+
+cudaError_t launch_indexer_prefill_mma(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
+                                       const float *sk, int HI, int dI, int row_begin, int n_rows, float *scores,
+                                       int64_t ld, cudaStream_t stream) {
+    if (n_rows == 0) return cudaSuccess;
+    const int key_tiles = (row_begin + n_rows + kKeysPerCta - 1) / kKeysPerCta;
+    const bool ok = dispatch_shape(HI, dI, [&](auto di, auto nt) {
+        constexpr int DI = decltype(di)::value, NT = decltype(nt)::value;
+        constexpr int QB = prefill_qb<DI, NT>();
+        const dim3 grid(key_tiles, (n_rows + QB - 1) / QB);
+        indexer_prefill_mma_kernel<DI, NT><<<grid, 256, 0, stream>>>(q8, sq, w, k8, sk, HI, row_begin, n_rows,
+                                                                    scores, ld);
+        return true;
+    });
+    return ok ? cudaGetLastError() : cudaErrorInvalidValue;
+}
+
+cudaError_t launch_indexer_decode(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8c,
+                                  const float *skc, const int32_t *block_table, int max_pages, int num_pages,
+                                  const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI, float *scores,
+                                  int64_t ld, cudaStream_t stream) {
+    if (B == 0 || max_seq_len == 0) return cudaSuccess;
+    const dim3 grid((max_seq_len + kKeysPerCta - 1) / kKeysPerCta, B);
+    const bool ok = dispatch_shape(HI, dI, [&](auto di, auto nt) {
+        constexpr int DI = decltype(di)::value, NT = decltype(nt)::value;
+        indexer_decode_mma_kernel<DI, NT><<<grid, 256, 0, stream>>>(
+            q8, sq, w, k8c, skc, block_table, max_pages, num_pages, seq_lens, max_seq_len, HI, scores, ld);
+        return true;
+    });
+    return ok ? cudaGetLastError() : cudaErrorInvalidValue;
+}
+
+}  // namespace dsa

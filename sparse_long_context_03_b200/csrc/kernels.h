@@ -1,0 +1,36 @@
+// kernels.h -- internal launchers behind the C ABI (not part of the ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace dsa {
+
+// indexer_mma.cu
+bool indexer_shape_supported(int HI, int dI);
+cudaError_t launch_indexer_prefill_mma(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
+                                       const float *sk, int HI, int dI, int row_begin, int n_rows, float *scores,
+                                       int64_t ld, cudaStream_t stream);
+cudaError_t launch_indexer_decode(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8c,
+                                  const float *skc, const int32_t *block_table, int max_pages, int num_pages,
+                                  const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI, float *scores,
+                                  int64_t ld, cudaStream_t stream);
+
+// topk.cu
+size_t topk_workspace_bytes(int n_rows, int max_len, int k);
+cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_rows, const int32_t *row_len,
+                        int max_len, int k, int32_t *idx, void *ws, size_t ws_bytes, cudaStream_t stream);
+
+// attention.cu
+bool attention_shape_supported(int Hq, int Hkv, int D);
+cudaError_t launch_sparse_prefill(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const int32_t *idx,
+                                  int row_begin, int n_rows, int Hq, int Hkv, int D, int k, float sm_scale,
+                                  uint16_t *O, float *lse, cudaStream_t stream);
+size_t decode_attention_workspace_bytes(int B, int Hq, int Hkv, int D, int k);
+cudaError_t launch_sparse_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                                 const int32_t *block_table, int max_pages, int num_pages, const int32_t *seq_lens,
+                                 const int32_t *idx, int B, int Hq, int Hkv, int D, int k, float sm_scale,
+                                 void *ws, size_t ws_bytes, uint16_t *out, float *lse, cudaStream_t stream);
+
+}  // namespace dsa

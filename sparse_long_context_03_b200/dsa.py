@@ -1,0 +1,247 @@
+"""ctypes binding of ``libdsa.so`` (C ABI in ``include/dsa.h``).
+
+Argument marshalling only: each function checks dtypes and shapes of the
+torch tensors it is given, passes their device pointers and the current CUDA
+stream to the C entry point of the same name, and raises ``DSAError`` on a
+non-zero status.  Every arithmetic step runs in the library's CUDA kernels;
+there is no other implementation behind these names, and a missing library
+raises instead of falling back to anything.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsa.so")
+PAGE_SIZE = 64
+
+_lib = None
+
+
+class DSAError(RuntimeError):
+    pass
+
+
+_P, _I, _I64, _SZ, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+
+_SIGNATURES = {
+    "dsa_status_string": ([_I], ctypes.c_char_p),
+    "dsa_version": ([], _I),
+    "dsa_last_error_string": ([], ctypes.c_char_p),
+    "dsa_indexer_scores": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P], _I),
+    "dsa_topk_workspace_size": ([_I, _I, _I], _SZ),
+    "dsa_topk": ([_P, _I64, _I, _I, _P, _I, _I, _P, _P, _SZ, _P], _I),
+    "dsa_sparse_gqa_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P], _I),
+    "dsa_decode_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
+    "dsa_sparse_gqa_decode": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _I,
+                               _I, _I, _I, _I, _I, _I, _I, _F, _P, _SZ, _P, _P, _P], _I),
+    "dsa_decode_indexer_scores": ([_P, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _I, _P, _I64, _P], _I),
+    "dsa_decode_attention_workspace_size": ([_I, _I, _I, _I, _I], _SZ),
+    "dsa_sparse_gqa_decode_attention": ([_P, _P, _P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _I, _F,
+                                         _P, _SZ, _P, _P, _P], _I),
+}
+
+
+def lib():
+    """Open libdsa.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise DSAError(f"{LIB_PATH} is missing; build it with `python -m sparse_long_context_03_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = handle
+    return _lib
+
+
+def exported_symbols():
+    return list(_SIGNATURES)
+
+
+def version() -> int:
+    return lib().dsa_version()
+
+
+def status_string(code: int) -> str:
+    return lib().dsa_status_string(int(code)).decode()
+
+
+def _check(code: int, name: str):
+    if code != 0:
+        err = lib().dsa_last_error_string().decode()
+        raise DSAError(f"{name}: {status_string(code)}" + (f" ({err})" if err else ""))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _need(t, dtype, ndim, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name}: expected {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+
+
+# ---------------------------------------------------------------------------
+# prefill
+# ---------------------------------------------------------------------------
+
+def indexer_scores(q8, q_scale, w, k8, k_scale, row_begin, n_rows, scores, stream=None):
+    """dsa_indexer_scores: rows [row_begin, row_begin+n_rows) of the causal
+    lightning-indexer score matrix into ``scores`` [n_rows, ld] float32."""
+    _need(q8, torch.uint8, 3, "q8")
+    _need(k8, torch.uint8, 2, "k8")
+    _need(scores, torch.float32, 2, "scores")
+    L, HI, dI = q8.shape
+    _check(lib().dsa_indexer_scores(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), L, HI, dI,
+                                    int(row_begin), int(n_rows), _ptr(scores), scores.stride(0), _stream(stream)),
+           "dsa_indexer_scores")
+
+
+def topk_workspace_size(n_rows, max_len, k) -> int:
+    return int(lib().dsa_topk_workspace_size(int(n_rows), int(max_len), int(k)))
+
+
+def topk(scores, row_begin, n_rows, k, idx, row_len=None, max_len=None, ws=None, stream=None):
+    """dsa_topk: per-row top-k (ascending indices, -1 padded) into idx [n_rows, k]."""
+    _need(scores, torch.float32, 2, "scores")
+    _need(idx, torch.int32, 2, "idx")
+    if max_len is None:
+        max_len = scores.shape[1] if row_len is not None else row_begin + n_rows
+    need = topk_workspace_size(n_rows, max_len, k)
+    ws_bytes = 0
+    if need:
+        if ws is None:
+            raise DSAError(f"dsa_topk needs a {need}-byte workspace")
+        ws_bytes = ws.numel() * ws.element_size()
+    _check(lib().dsa_topk(_ptr(scores), scores.stride(0), int(row_begin), int(n_rows), _ptr(row_len), int(max_len),
+                          int(k), _ptr(idx), _ptr(ws), ws_bytes, _stream(stream)), "dsa_topk")
+
+
+def sparse_gqa_prefill(Q, K, V, idx, row_begin, n_rows, k, sm_scale, O, lse=None, stream=None):
+    """dsa_sparse_gqa_prefill: attention of query rows [row_begin, row_begin+n_rows)
+    over their selected keys.  Q/O [n_rows,Hq,D] bf16, K/V [L,Hkv,D] bf16."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (O, "O")):
+        _need(t, torch.bfloat16, 3, n)
+    _need(idx, torch.int32, 2, "idx")
+    Hq, D = Q.shape[1], Q.shape[2]
+    Hkv = K.shape[1]
+    _check(lib().dsa_sparse_gqa_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), int(row_begin), int(n_rows), Hq, Hkv,
+                                        D, int(k), float(sm_scale), _ptr(O), _ptr(lse), _stream(stream)),
+           "dsa_sparse_gqa_prefill")
+
+
+class PrefillPlan:
+    """Buffers for a chunked prefill of one sequence (query-row chunks bound
+    the size of the score matrix, as the chunked indexer of report section
+    5.2.1 does).  The score buffer is [chunk_rows, ld] float32."""
+
+    def __init__(self, L, HI, dI, Hq, Hkv, D, k, chunk_rows=None, device="cuda", score_budget_bytes=4 << 30):
+        self.L, self.HI, self.dI, self.Hq, self.Hkv, self.D, self.k = L, HI, dI, Hq, Hkv, D, k
+        self.ld = (L + 3) // 4 * 4
+        if chunk_rows is None:
+            chunk_rows = max(1, min(L, score_budget_bytes // (4 * self.ld)))
+        self.chunk_rows = int(chunk_rows)
+        self.scores = torch.empty(self.chunk_rows, self.ld, dtype=torch.float32, device=device)
+        self.idx = torch.empty(L, k, dtype=torch.int32, device=device)
+        need = topk_workspace_size(self.chunk_rows, L, k)
+        self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=device) if need else None
+
+    def chunks(self):
+        for r0 in range(0, self.L, self.chunk_rows):
+            yield r0, min(self.chunk_rows, self.L - r0)
+
+
+def prefill_forward(plan: PrefillPlan, q8, sq, w, k8, sk, Q, K, V, O, sm_scale=None, lse=None, stream=None):
+    """Whole DSA prefill of one sequence: for each chunk of query rows, the
+    indexer scores then the top-k; then the sparse attention of every row.
+    Writes plan.idx [L,k] and O [L,Hq,D] (lse [L,Hq] if given)."""
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(plan.D)
+    for r0, n in plan.chunks():
+        indexer_scores(q8, sq, w, k8, sk, r0, n, plan.scores[:n], stream=stream)
+        topk(plan.scores[:n], r0, n, plan.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws, stream=stream)
+    sparse_gqa_prefill(Q, K, V, plan.idx, 0, plan.L, plan.k, sm_scale, O, lse, stream=stream)
+
+
+# ---------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------
+
+def decode_workspace_size(B, max_seq_len, Hq, Hkv, D, k) -> int:
+    return int(lib().dsa_decode_workspace_size(int(B), int(max_seq_len), int(Hq), int(Hkv), int(D), int(k)))
+
+
+def decode_attention_workspace_size(B, Hq, Hkv, D, k) -> int:
+    return int(lib().dsa_decode_attention_workspace_size(int(B), int(Hq), int(Hkv), int(D), int(k)))
+
+
+def decode_indexer_scores(q8, q_scale, w, k8_cache, k_scale_cache, block_table, seq_lens, max_seq_len, scores,
+                          stream=None):
+    _need(q8, torch.uint8, 3, "q8")
+    _need(k8_cache, torch.uint8, 3, "k8_cache")
+    _need(block_table, torch.int32, 2, "block_table")
+    _need(scores, torch.float32, 2, "scores")
+    B, HI, dI = q8.shape
+    _check(lib().dsa_decode_indexer_scores(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8_cache), _ptr(k_scale_cache),
+                                           _ptr(block_table), block_table.shape[1], k8_cache.shape[0],
+                                           _ptr(seq_lens), int(max_seq_len), B, HI, dI, _ptr(scores),
+                                           scores.stride(0), _stream(stream)), "dsa_decode_indexer_scores")
+
+
+def sparse_gqa_decode_attention(q, k_cache, v_cache, block_table, seq_lens, idx, k, sm_scale, ws, out, lse=None,
+                                stream=None):
+    _need(q, torch.bfloat16, 3, "q")
+    _need(k_cache, torch.bfloat16, 4, "k_cache")
+    _need(v_cache, torch.bfloat16, 4, "v_cache")
+    _need(out, torch.bfloat16, 3, "out")
+    B, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    _check(lib().dsa_sparse_gqa_decode_attention(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                                 block_table.shape[1], k_cache.shape[0], _ptr(seq_lens), _ptr(idx),
+                                                 B, Hq, Hkv, D, int(k), float(sm_scale), _ptr(ws),
+                                                 ws.numel() * ws.element_size(), _ptr(out), _ptr(lse),
+                                                 _stream(stream)), "dsa_sparse_gqa_decode_attention")
+
+
+def sparse_gqa_decode(q, q8, q_scale, w, k8_cache, k_scale_cache, k_cache, v_cache, block_table, seq_lens,
+                      max_seq_len, k, sm_scale, ws, out, idx_out=None, stream=None):
+    """dsa_sparse_gqa_decode: indexer -> top-k -> attention for one new token per sequence."""
+    _need(q, torch.bfloat16, 3, "q")
+    _need(q8, torch.uint8, 3, "q8")
+    _need(k_cache, torch.bfloat16, 4, "k_cache")
+    _need(block_table, torch.int32, 2, "block_table")
+    _need(out, torch.bfloat16, 3, "out")
+    B, Hq, D = q.shape
+    HI, dI = q8.shape[1], q8.shape[2]
+    Hkv = k_cache.shape[2]
+    _check(lib().dsa_sparse_gqa_decode(_ptr(q), _ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8_cache),
+                                       _ptr(k_scale_cache), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                       block_table.shape[1], k_cache.shape[0], _ptr(seq_lens), int(max_seq_len), B,
+                                       Hq, Hkv, D, HI, dI, int(k), float(sm_scale), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _ptr(out), _ptr(idx_out), _stream(stream)),
+           "dsa_sparse_gqa_decode")

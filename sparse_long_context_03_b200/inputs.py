@@ -209,6 +209,8 @@ def decode_inputs(cfg: Config, device="cpu", seed: int | None = None, B: int | N
     The query token sits at position seq_len-1, already in the cache.
     """
     g = _gen(device, cfg.seed if seed is None else seed)
+    if seq_lens is not None:
+        B = len(seq_lens)
     B = cfg.B if B is None else B
     lo = cfg.len_lo if len_lo is None else len_lo
     hi = cfg.len_hi if len_hi is None else len_hi

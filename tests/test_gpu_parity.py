@@ -1,0 +1,383 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Every case draws seeded inputs, runs the library on a B200 and the oracle on
+the host on the same bytes, and compares with the criteria in
+parity_helpers.  Small cases cover whole matrices (several tiles and a
+ragged tail); the full-size workloads run in the benchmark's launch
+configuration and are compared on sampled rows.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_helpers import (check_attention, check_scores, check_topk_row, check_topk_structure)
+from sparse_long_context_03_b200 import dsa, inputs
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def H(t):
+    return inputs.to_numpy_bits(t)
+
+
+def _gpu(d):
+    return {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+def gpu_scores(d, row_begin, n_rows, L):
+    ld = (L + 3) // 4 * 4
+    out = torch.full((n_rows, ld), float("nan"), dtype=torch.float32, device=DEV)
+    dsa.indexer_scores(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], row_begin, n_rows, out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+# ----------------------------------------------------------------------------
+# indexer
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("row_begin,n_rows", [(0, 512), (200, 137), (511, 1)])
+def test_indexer_tiny_matches_oracle(row_begin, n_rows):
+    cfg = inputs.config(0)
+    d = inputs.prefill_inputs(cfg)
+    ref = oracle.indexer(*(H(d[k]) for k in ("q8", "sq", "w", "k8", "sk")), row_begin=row_begin, n_rows=n_rows)
+    got = gpu_scores(_gpu(d), row_begin, n_rows, cfg.L)
+    for r in range(n_rows):
+        t = row_begin + r
+        check_scores(got[r, : t + 1], ref[r, : t + 1], f"row {t}")
+
+
+@pytest.mark.parametrize("HI,dI,L", [(32, 64, 700), (4, 32, 300), (64, 128, 260), (16, 64, 333), (8, 32, 129)])
+def test_indexer_exact_inputs_bit_exact(HI, dI, L):
+    d = inputs.exact_indexer_inputs(L, HI, dI, seed=100 + HI + dI)
+    ref = oracle.indexer(*(H(d[k]) for k in ("q8", "sq", "w", "k8", "sk")))
+    got = gpu_scores(_gpu(d), 0, L, L)
+    tri = np.tril(np.ones((L, L), bool))
+    assert np.array_equal(got[:, :L][tri].astype(np.float64), ref[tri])
+
+
+def test_indexer_signed_weights():
+    cfg = inputs.config(0)
+    d = inputs.prefill_inputs(cfg, L=300, seed=44)
+    g = torch.Generator().manual_seed(3)
+    d["w"] = torch.randn(300, cfg.HI, generator=g)
+    ref = oracle.indexer(*(H(d[k]) for k in ("q8", "sq", "w", "k8", "sk")))
+    got = gpu_scores(_gpu(d), 0, 300, 300)
+    assert (ref[np.tril(np.ones((300, 300), bool))] < 0).any()
+    for t in range(300):
+        check_scores(got[t, : t + 1], ref[t, : t + 1], f"row {t}")
+
+
+# ----------------------------------------------------------------------------
+# top-k
+# ----------------------------------------------------------------------------
+
+def gpu_topk(scores_np, k, row_begin=0, row_len=None, max_len=None):
+    n_rows, w = scores_np.shape
+    ld = (w + 3) // 4 * 4
+    s = torch.zeros(n_rows, ld, dtype=torch.float32)
+    s[:, :w] = torch.from_numpy(scores_np)
+    s = s.to(DEV)
+    idx = torch.full((n_rows, k), -7, dtype=torch.int32, device=DEV)
+    rl = None if row_len is None else torch.as_tensor(row_len, dtype=torch.int32, device=DEV)
+    if max_len is None:
+        max_len = w if row_len is not None else row_begin + n_rows
+    need = dsa.topk_workspace_size(n_rows, max_len, k)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=DEV) if need else None
+    dsa.topk(s, row_begin, n_rows, k, idx, row_len=rl, max_len=max_len, ws=ws)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy()
+
+
+@pytest.mark.parametrize("k", [1, 7, 64, 300])
+def test_topk_causal_rows_bit_exact(k):
+    n_rows = 600
+    x = inputs.tie_heavy_scores(n_rows, n_rows, seed=10 + k).numpy()
+    got = gpu_topk(x, k)
+    ref = oracle.causal_topk(x.astype(np.float64), 0, k)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("k", [1, 64, 2048])
+def test_topk_row_lengths_bit_exact(k):
+    lens = [0, 1, 2, k - 1, k, k + 1, 2 * k + 3, 5000, 20000, 65537, 3, 100000]
+    width = max(lens)
+    x = inputs.tie_heavy_scores(len(lens), width, seed=77 + k).numpy()
+    got = gpu_topk(x, k, row_len=lens)
+    ref = oracle.topk(x.astype(np.float64), lens, k)
+    assert np.array_equal(got, ref)
+
+
+def test_topk_chunk_offset_and_determinism():
+    x = inputs.tie_heavy_scores(97, 3000, seed=5).numpy()
+    a = gpu_topk(x, 256, row_begin=2903, max_len=3000)
+    b = gpu_topk(x, 256, row_begin=2903, max_len=3000)
+    assert np.array_equal(a, b)
+    ref = oracle.topk(x.astype(np.float64), np.arange(2904, 3001), 256)
+    assert np.array_equal(a, ref)
+
+
+def test_topk_signed_zeros_and_all_equal():
+    x = np.zeros((3, 100), np.float32)
+    x[0, ::2] = -0.0
+    x[1, :] = 0.5
+    x[2, :] = -3.0
+    x[2, 50] = -0.0
+    got = gpu_topk(x, 10, row_len=[100, 100, 100])
+    assert list(got[0]) == list(range(10))
+    assert list(got[1]) == list(range(10))
+    assert list(got[2]) == [0, 1, 2, 3, 4, 5, 6, 7, 8, 50]
+
+
+# ----------------------------------------------------------------------------
+# whole prefill chain, small
+# ----------------------------------------------------------------------------
+
+def run_prefill(cfg, d, chunk_rows=None, want_rows=(), lse=True):
+    """Run the chunked prefill exactly as the benchmark does; also copy out
+    the score rows listed in want_rows as each chunk is produced."""
+    L = d["q8"].shape[0]
+    plan = dsa.PrefillPlan(L, cfg.HI, cfg.dI, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, chunk_rows=chunk_rows)
+    O = torch.empty(L, cfg.Hq, cfg.D, dtype=torch.bfloat16, device=DEV)
+    lse_t = torch.empty(L, cfg.Hq, dtype=torch.float32, device=DEV) if lse else None
+    want = sorted(want_rows)
+    rows = {}
+    for r0, n in plan.chunks():
+        dsa.indexer_scores(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], r0, n, plan.scores[:n])
+        for t in want:
+            if r0 <= t < r0 + n:
+                rows[t] = plan.scores[t - r0, : t + 1].cpu().numpy()
+        dsa.topk(plan.scores[:n], r0, n, cfg.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws)
+    dsa.sparse_gqa_prefill(d["Q"], d["K"], d["V"], plan.idx, 0, L, cfg.k, cfg.sm_scale, O, lse_t)
+    torch.cuda.synchronize()
+    return plan, O, lse_t, rows
+
+
+def test_prefill_chain_tiny_full():
+    cfg = inputs.config(0)
+    d = inputs.prefill_inputs(cfg)
+    plan, O, lse, _ = run_prefill(cfg, _gpu(d), chunk_rows=200)
+    h = {k: H(v) for k, v in d.items()}
+    I = oracle.indexer(h["q8"], h["sq"], h["w"], h["k8"], h["sk"])
+    ref_idx = oracle.causal_topk(I, 0, cfg.k)
+    gidx = plan.idx.cpu().numpy()
+    for t in range(cfg.L):
+        check_topk_row(gidx[t], ref_idx[t], I[t], t + 1, cfg.k, f"row {t}")
+    Oref, lref = oracle.sparse_attention(h["Q"], h["K"], h["V"], ref_idx, 0, cfg.sm_scale)
+    same = np.all(gidx == ref_idx, axis=1)
+    Og = O.float().cpu().numpy()
+    check_attention(Og[same], Oref[same], lse.cpu().numpy()[same], lref[same], "chain")
+    # the attention kernel alone on the oracle's index sets, every row
+    O2 = torch.empty_like(O)
+    l2 = torch.empty_like(lse)
+    dsa.sparse_gqa_prefill(_gpu(d)["Q"], _gpu(d)["K"], _gpu(d)["V"], torch.from_numpy(ref_idx).to(DEV), 0, cfg.L,
+                           cfg.k, cfg.sm_scale, O2, l2)
+    torch.cuda.synchronize()
+    check_attention(O2.float().cpu().numpy(), Oref, l2.cpu().numpy(), lref, "attention on oracle idx")
+
+
+def test_prefill_chain_exact_inputs_bit_exact_indices():
+    cfg = inputs.config(1, k=64)
+    L = 900
+    d = inputs.exact_indexer_inputs(L, cfg.HI, cfg.dI, seed=9, key_pool=24)
+    g = torch.Generator().manual_seed(1)
+    for name, Hh in (("Q", cfg.Hq), ("K", cfg.Hkv), ("V", cfg.Hkv)):
+        d[name] = (torch.randn(L, Hh, cfg.D, generator=g) * 0.5).to(torch.bfloat16)
+    plan, O, lse, _ = run_prefill(cfg, _gpu(d), chunk_rows=256)
+    h = {k: H(v) for k, v in d.items()}
+    I = oracle.indexer(h["q8"], h["sq"], h["w"], h["k8"], h["sk"])
+    ref_idx = oracle.causal_topk(I, 0, cfg.k)
+    assert np.array_equal(plan.idx.cpu().numpy(), ref_idx)
+    Oref, lref = oracle.sparse_attention(h["Q"], h["K"], h["V"], ref_idx, 0, cfg.sm_scale)
+    check_attention(O.float().cpu().numpy(), Oref, lse.cpu().numpy(), lref, "exact chain")
+
+
+# ----------------------------------------------------------------------------
+# attention edge cases
+# ----------------------------------------------------------------------------
+
+def _dense_causal(Qd, Kd, Vd, sm):
+    L, Hq, D = Qd.shape
+    G = Hq // Kd.shape[1]
+    O = np.zeros_like(Qd)
+    for h in range(Hq):
+        lg = sm * Qd[:, h] @ Kd[:, h // G].T
+        lg[np.triu(np.ones((L, L), bool), 1)] = -np.inf
+        lg -= lg.max(axis=1, keepdims=True)
+        p = np.exp(lg)
+        O[:, h] = (p / p.sum(axis=1, keepdims=True)) @ Vd[:, h // G]
+    return O
+
+
+@pytest.mark.parametrize("Hq,Hkv,D", [(8, 2, 64), (32, 4, 128), (8, 8, 64), (16, 2, 128)])
+def test_attention_full_budget_equals_dense(Hq, Hkv, D):
+    L, k = 150, 160
+    g = torch.Generator().manual_seed(Hq + D)
+    Q = torch.randn(L, Hq, D, generator=g).to(torch.bfloat16)
+    K = torch.randn(L, Hkv, D, generator=g).to(torch.bfloat16)
+    V = torch.randn(L, Hkv, D, generator=g).to(torch.bfloat16)
+    idx = np.full((L, k), -1, np.int32)
+    for t in range(L):
+        idx[t, : t + 1] = np.arange(t + 1)
+    O = torch.empty(L, Hq, D, dtype=torch.bfloat16, device=DEV)
+    sm = 1 / math.sqrt(D)
+    dsa.sparse_gqa_prefill(Q.to(DEV), K.to(DEV), V.to(DEV), torch.from_numpy(idx).to(DEV), 0, L, k, sm, O)
+    torch.cuda.synchronize()
+    ref = _dense_causal(Q.double().numpy(), K.double().numpy(), V.double().numpy(), sm)
+    check_attention(O.float().cpu().numpy(), ref, what="dense")
+
+
+def test_attention_skips_invalid_entries_and_empty_rows():
+    L, Hq, Hkv, D, k = 40, 8, 2, 64, 16
+    g = torch.Generator().manual_seed(8)
+    Q = torch.randn(L, Hq, D, generator=g).to(torch.bfloat16)
+    K = torch.randn(L, Hkv, D, generator=g).to(torch.bfloat16)
+    V = torch.randn(L, Hkv, D, generator=g).to(torch.bfloat16)
+    idx = np.full((L, k), -1, np.int32)
+    for t in range(1, L):
+        sel = np.arange(0, t + 1, 3)[:k]
+        idx[t, : len(sel)] = sel
+    idx[30, 5] = 35          # beyond t: must be skipped
+    idx[31, 2] = 1 << 30     # far out of range: must be skipped
+    idx[0, :] = -1           # no valid entry: O = 0, lse = -inf
+    O = torch.empty(L, Hq, D, dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty(L, Hq, dtype=torch.float32, device=DEV)
+    dsa.sparse_gqa_prefill(Q.to(DEV), K.to(DEV), V.to(DEV), torch.from_numpy(idx).to(DEV), 0, L, k, 0.125, O, lse)
+    torch.cuda.synchronize()
+    Oref, lref = oracle.sparse_attention(H(Q), H(K), H(V), idx, 0, 0.125)
+    check_attention(O.float().cpu().numpy(), Oref, lse.cpu().numpy(), lref, "invalid entries")
+    assert np.all(O[0].float().cpu().numpy() == 0) and np.all(np.isneginf(lse[0].cpu().numpy()))
+
+
+# ----------------------------------------------------------------------------
+# decode
+# ----------------------------------------------------------------------------
+
+def run_decode(cfg, d, k):
+    B = d["q"].shape[0]
+    need = dsa.decode_workspace_size(B, d["max_seq_len"], cfg.Hq, cfg.Hkv, cfg.D, k)
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    out = torch.empty(B, cfg.Hq, cfg.D, dtype=torch.bfloat16, device=DEV)
+    idx = torch.full((B, k), -7, dtype=torch.int32, device=DEV)
+    dsa.sparse_gqa_decode(d["q"], d["q8"], d["sq"], d["w"], d["k8_cache"], d["sk_cache"], d["k_cache"],
+                          d["v_cache"], d["block_table"], d["seq_lens"], d["max_seq_len"], k, cfg.sm_scale, ws,
+                          out, idx_out=idx)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), idx.cpu().numpy()
+
+
+def check_decode(cfg, dh, out, idx, k):
+    h = {kk: (H(v) if isinstance(v, torch.Tensor) else v) for kk, v in dh.items()}
+    I = oracle.decode_indexer(h["q8"], h["sq"], h["w"], h["k8_cache"], h["sk_cache"], h["block_table"],
+                              h["seq_lens"])
+    ref_idx = oracle.topk(I, h["seq_lens"], k)
+    for b in range(len(h["seq_lens"])):
+        check_topk_row(idx[b], ref_idx[b], I[b], int(h["seq_lens"][b]), k, f"seq {b}")
+    Oref, _ = oracle.decode_attention(h["q"], h["k_cache"], h["v_cache"], h["block_table"], h["seq_lens"],
+                                      ref_idx, cfg.sm_scale)
+    same = np.all(idx == ref_idx, axis=1)
+    check_attention(out[same], Oref[same], what="decode")
+    return I, ref_idx, Oref
+
+
+@pytest.mark.parametrize("cfg_id,lens,k", [
+    (0, [1, 63, 64, 65, 300, 1000], 64),
+    (3, [1, 64, 2047, 2048, 2049, 5000, 70000], 2048),
+])
+def test_decode_small_matches_oracle(cfg_id, lens, k):
+    cfg = inputs.config(cfg_id)
+    d = inputs.decode_inputs(cfg, seq_lens=lens, seed=50 + cfg_id)
+    out, idx = run_decode(cfg, _gpu(d), k)
+    I, ref_idx, Oref = check_decode(cfg, d, out, idx, k)
+    # stage 1 alone: scores through the block table
+    g = _gpu(d)
+    ld = (d["max_seq_len"] + 3) // 4 * 4
+    sc = torch.zeros(len(lens), ld, dtype=torch.float32, device=DEV)
+    dsa.decode_indexer_scores(g["q8"], g["sq"], g["w"], g["k8_cache"], g["sk_cache"], g["block_table"],
+                              g["seq_lens"], d["max_seq_len"], sc)
+    # stage 3 alone on the oracle's index sets
+    ws = torch.empty(dsa.decode_attention_workspace_size(len(lens), cfg.Hq, cfg.Hkv, cfg.D, k), dtype=torch.uint8,
+                     device=DEV)
+    o3 = torch.empty(len(lens), cfg.Hq, cfg.D, dtype=torch.bfloat16, device=DEV)
+    l3 = torch.empty(len(lens), cfg.Hq, dtype=torch.float32, device=DEV)
+    dsa.sparse_gqa_decode_attention(g["q"], g["k_cache"], g["v_cache"], g["block_table"], g["seq_lens"],
+                                    torch.from_numpy(ref_idx).to(DEV), k, cfg.sm_scale, ws, o3, l3)
+    torch.cuda.synchronize()
+    scn = sc.cpu().numpy()
+    for b, n in enumerate(lens):
+        check_scores(scn[b, :n], I[b, :n], f"decode scores seq {b}")
+    h = {kk: (H(v) if isinstance(v, torch.Tensor) else v) for kk, v in d.items()}
+    Oref2, lref2 = oracle.decode_attention(h["q"], h["k_cache"], h["v_cache"], h["block_table"], h["seq_lens"],
+                                           ref_idx, cfg.sm_scale)
+    check_attention(o3.float().cpu().numpy(), Oref2, l3.cpu().numpy(), lref2, "decode attention stage")
+
+
+# ----------------------------------------------------------------------------
+# full-size workloads, sampled rows, benchmark launch configuration
+# ----------------------------------------------------------------------------
+
+def _sample_rows(L, k, extra, seed):
+    rng = np.random.default_rng(seed)
+    rows = {0, k - 2, k - 1, k, k + 1, L // 2 + 3, L - 1} | set(int(x) for x in rng.integers(0, L, 3)) | set(extra)
+    return sorted(r for r in rows if 0 <= r < L)
+
+
+@pytest.mark.parametrize("cfg_id", [1, 2, 4])
+def test_full_size_prefill_sampled_rows(cfg_id):
+    cfg = inputs.config(cfg_id)
+    d = inputs.prefill_inputs(cfg, device=DEV)
+    extra = []
+    if cfg.multimodal:  # frame / text boundaries
+        P = inputs.PERIOD
+        extra = [P * 7 + 4095, P * 7 + 4096, P * 7 + 4159, P * 20 + 256]
+    rows = _sample_rows(cfg.L, cfg.k, extra, seed=cfg_id)
+    plan, O, lse, got_rows = run_prefill(cfg, d, want_rows=rows)
+    h = {kk: H(d[kk]) for kk in ("q8", "sq", "w", "k8", "sk")}
+    Kh, Vh = H(d["K"]), H(d["V"])
+    sel = torch.tensor(rows, device=DEV)
+    gidx = plan.idx[sel].cpu().numpy()
+    Og, lg = O[sel].float().cpu().numpy(), lse[sel].cpu().numpy()
+    Qh = H(d["Q"][sel])
+    for i, t in enumerate(rows):
+        I = oracle.indexer(h["q8"], h["sq"], h["w"], h["k8"], h["sk"], row_begin=t, n_rows=1)[0]
+        check_scores(got_rows[t], I, f"cfg{cfg_id} row {t}")
+        ref_idx = oracle.topk(I[None, :], [t + 1], cfg.k)
+        check_topk_row(gidx[i], ref_idx[0], I, t + 1, cfg.k, f"cfg{cfg_id} row {t}")
+        Oref, lref = oracle.sparse_attention(Qh[i:i + 1], Kh, Vh, ref_idx, t, cfg.sm_scale)
+        if np.array_equal(gidx[i], ref_idx[0]):
+            check_attention(Og[i:i + 1], Oref, lg[i:i + 1], lref, f"cfg{cfg_id} row {t}")
+        else:
+            O1 = torch.empty(1, cfg.Hq, cfg.D, dtype=torch.bfloat16, device=DEV)
+            dsa.sparse_gqa_prefill(d["Q"][t:t + 1], d["K"], d["V"], torch.from_numpy(ref_idx).to(DEV), t, 1, cfg.k,
+                                   cfg.sm_scale, O1)
+            torch.cuda.synchronize()
+            check_attention(O1.float().cpu().numpy(), Oref, what=f"cfg{cfg_id} row {t} (oracle idx)")
+    check_index_structure_on_device(plan.idx, 0, cfg.k)
+
+
+def check_index_structure_on_device(idx, row_begin, k, row_len=None, step=8192):
+    """Every row: count = min(k, n), ascending, within [0, n), -1 padded."""
+    L = idx.shape[0]
+    ar = torch.arange(k, device=idx.device)
+    for r0 in range(0, L, step):
+        blk = idx[r0:r0 + step]
+        r = torch.arange(r0, r0 + blk.shape[0], device=idx.device)
+        n = (row_begin + r + 1) if row_len is None else row_len[r0:r0 + step]
+        cnt = torch.clamp(n, max=k)
+        valid = blk >= 0
+        assert torch.equal(valid, ar[None, :] < cnt[:, None]), "count / padding"
+        assert bool(((blk[:, 1:] > blk[:, :-1]) | ~valid[:, 1:]).all()), "ascending"
+        assert bool((torch.where(valid, blk, -1) < n[:, None]).all()), "range"
+        assert bool((blk[~valid] == -1).all()), "padding value"
+
+
+def test_full_size_decode_all_sequences():
+    cfg = inputs.config(3)
+    d = inputs.decode_inputs(cfg, device=DEV)
+    out, idx = run_decode(cfg, d, cfg.k)
+    check_decode(cfg, d, out, idx, cfg.k)
