@@ -67,6 +67,11 @@ DSA_API const char *dsa_status_string(dsa_status_t s);
 DSA_API int dsa_version(void);
 /* Text of the last CUDA error seen by a dsa_* call on this thread ("" if none). */
 DSA_API const char *dsa_last_error_string(void);
+/* Diagnostic, not for the hot path: synchronises the current device, then
+ * returns DSA_ERR_TIMEOUT if a kernel's bounded wait on an on-chip barrier
+ * expired since the last call (the kernel then wrote incomplete results and
+ * exited cleanly), DSA_OK otherwise.  Clears the flag. */
+DSA_API dsa_status_t dsa_check_device_error(void);
 
 /* ------------------------------------------------------------------------
  * Lightning-indexer scores (prefill), one chunk of query rows.
@@ -84,6 +89,8 @@ DSA_API const char *dsa_last_error_string(void);
  *   scores   [n_rows, ld_scores] float; row r holds query t = row_begin + r;
  *            columns 0..t are written, columns > t are left unspecified.
  *            ld_scores >= row_begin + n_rows and ld_scores % 4 == 0.
+ *   q8, k8 must be 16-byte aligned (they are read by the tensor-memory
+ *   accelerator).
  * Supported: dI in {32, 64, 128}; HI in {4, 8, 16, 32, 64}.
  * All scale factors must be positive (they commute with the ReLU).
  * ------------------------------------------------------------------------ */

@@ -60,6 +60,13 @@ int dsa_version(void) { return DSA_VERSION; }
 
 const char *dsa_last_error_string(void) { return g_last_error; }
 
+dsa_status_t dsa_check_device_error(void) {
+    unsigned int flag = 0;
+    cudaError_t e = dsa::indexer_tc_take_error(&flag);
+    if (e != cudaSuccess) return cuda_status(e);
+    return flag ? DSA_ERR_TIMEOUT : DSA_OK;
+}
+
 dsa_status_t dsa_indexer_scores(const uint8_t *q8, const float *q_scale, const float *w, const uint8_t *k8,
                                 const float *k_scale, int L, int HI, int dI, int row_begin, int n_rows,
                                 float *scores, int64_t ld_scores, void *stream) {
@@ -68,6 +75,10 @@ dsa_status_t dsa_indexer_scores(const uint8_t *q8, const float *q_scale, const f
     if (n_rows == 0) return DSA_OK;
     if (!q8 || !q_scale || !w || !k8 || !k_scale || !scores) return DSA_ERR_INVALID_ARG;
     if (ld_scores < (int64_t)row_begin + n_rows || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(q8) | reinterpret_cast<uintptr_t>(k8)) % 16 != 0) return DSA_ERR_INVALID_ARG;
+    if (dsa::indexer_tc_supported(HI, dI))
+        return cuda_status(dsa::launch_indexer_prefill_tc(q8, q_scale, w, k8, k_scale, L, HI, dI, row_begin, n_rows,
+                                                          scores, ld_scores, as_stream(stream)));
     return cuda_status(dsa::launch_indexer_prefill_mma(q8, q_scale, w, k8, k_scale, HI, dI, row_begin, n_rows,
                                                        scores, ld_scores, as_stream(stream)));
 }

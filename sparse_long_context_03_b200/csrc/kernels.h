@@ -17,6 +17,13 @@ cudaError_t launch_indexer_decode(const uint8_t *q8, const float *sq, const floa
                                   const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI, float *scores,
                                   int64_t ld, cudaStream_t stream);
 
+// indexer_tc.cu
+bool indexer_tc_supported(int HI, int dI);
+cudaError_t launch_indexer_prefill_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
+                                      const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
+                                      float *scores, int64_t ld, cudaStream_t stream);
+cudaError_t indexer_tc_take_error(unsigned int *flag);
+
 // topk.cu
 size_t topk_workspace_bytes(int n_rows, int max_len, int k);
 cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_rows, const int32_t *row_len,

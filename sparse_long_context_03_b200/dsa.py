@@ -32,6 +32,7 @@ _SIGNATURES = {
     "dsa_status_string": ([_I], ctypes.c_char_p),
     "dsa_version": ([], _I),
     "dsa_last_error_string": ([], ctypes.c_char_p),
+    "dsa_check_device_error": ([], _I),
     "dsa_indexer_scores": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P], _I),
     "dsa_topk_workspace_size": ([_I, _I, _I], _SZ),
     "dsa_topk": ([_P, _I64, _I, _I, _P, _I, _I, _P, _P, _SZ, _P], _I),
@@ -71,6 +72,11 @@ def version() -> int:
 
 def status_string(code: int) -> str:
     return lib().dsa_status_string(int(code)).decode()
+
+
+def check_device_error():
+    """Synchronises; raises DSAError if a kernel's bounded wait expired."""
+    _check(lib().dsa_check_device_error(), "dsa_check_device_error")
 
 
 def _check(code: int, name: str):
