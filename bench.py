@@ -65,12 +65,23 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device="cuda") -> float:
+    """The slowest rank's time: every rank contributes its own device-timed value."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(cfg, rank: int) -> int:
+    """Each rank prefills its own independent sequence (weak scaling)."""
+    return cfg.seed + 7919 * rank
+
+
+def aggregate_tok_per_s(world: int, tokens_per_rank: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: tokens of all ranks over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (ms_max / 1e3)
 
 
 # ----------------------------------------------------------------------------
@@ -136,12 +147,13 @@ def causal_pairs(r0, n):
 
 
 class PrefillBench:
-    def __init__(self, cfg, seed, device):
+    def __init__(self, cfg, seed, device, chunk_rows=None):
         from sparse_long_context_03_b200 import dsa, inputs
         self.dsa = dsa
         self.cfg = cfg
         self.d = inputs.prefill_inputs(cfg, device=device, seed=seed)
-        self.plan = dsa.PrefillPlan(cfg.L, cfg.HI, cfg.dI, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, device=device)
+        self.plan = dsa.PrefillPlan(cfg.L, cfg.HI, cfg.dI, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, chunk_rows=chunk_rows,
+                                    device=device)
         self.O = torch.empty(cfg.L, cfg.Hq, cfg.D, dtype=torch.bfloat16, device=device)
         self.stream = torch.cuda.current_stream()
         self.chunks = list(self.plan.chunks())
@@ -412,6 +424,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--chunk-rows", type=int, default=None,
+                    help="query rows per indexer/top-k chunk (default: a 4 GiB score block)")
     args = ap.parse_args()
 
     if args.impl == "reference":
@@ -427,11 +441,11 @@ def main():
 
     pk, src = peaks()
     cfg = inputs.config(args.config)
-    pb = PrefillBench(cfg, seed=cfg.seed + 7919 * rank, device="cuda")
+    pb = PrefillBench(cfg, seed=rank_seed(cfg, rank), device="cuda", chunk_rows=args.chunk_rows)
     chunk_rows = pb.plan.chunk_rows
     ms, per, clocks = run_prefill_timed(pb, args.steps, args.warmup, world, local)
     ms_max = max_over_ranks(ms, world)
-    value = world * cfg.L * args.steps / (ms_max / 1e3)
+    value = aggregate_tok_per_s(world, cfg.L, args.steps, ms_max)
     stages = stage_roofline(per, pb, pk, src)
     dominant = max(stages, key=lambda k: stages[k]["ms_total"])
     dom = dict(stages[dominant])
@@ -443,7 +457,7 @@ def main():
         ems, h2d, d2h = run_prefill_e2e(pb, max(1, min(args.steps, 3)), 1)
         n_e2e = max(1, min(args.steps, 3))
         ems = max_over_ranks(ems, world)
-        e2e = {"value": world * cfg.L * n_e2e / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": aggregate_tok_per_s(world, cfg.L, n_e2e, ems), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ems / n_e2e}
 
     decode = None
@@ -451,7 +465,7 @@ def main():
         del pb
         torch.cuda.empty_cache()
         dcfg = inputs.config(3)
-        db = DecodeBench(dcfg, seed=dcfg.seed + 7919 * rank, device="cuda")
+        db = DecodeBench(dcfg, seed=rank_seed(dcfg, rank), device="cuda")
         us = 1e3 * max_over_ranks(run_decode_timed(db, max(args.steps, 20), max(args.warmup, 3)), world)
         byts = db.algorithmic_bytes()
         decode = {"workload": f"{dcfg.name}: B={db.B}, cached lengths U[{dcfg.len_lo},{dcfg.len_hi}] "

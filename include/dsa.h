@@ -112,7 +112,8 @@ DSA_API dsa_status_t dsa_indexer_scores(const uint8_t *q8, const float *q_scale,
  * indices of the largest scores, ties broken toward the lower index, -0.0 and
  * +0.0 equal.  Indices ascending, padded with -1.
  *   max_len  upper bound of every n_r (the host sizes grids with it);
- *            ld_scores >= max_len and ld_scores % 4 == 0.
+ *            ld_scores >= max_len and ld_scores % 4 == 0; scores 16-byte aligned.
+ * Supported: 1 <= k <= 40000 (a row's winners are staged in shared memory).
  *   ws       device workspace of at least dsa_topk_workspace_size() bytes
  *            (may be NULL when that size is 0).
  * ------------------------------------------------------------------------ */

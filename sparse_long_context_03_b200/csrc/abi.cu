@@ -95,6 +95,8 @@ dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, int row_begin, int
     if (n_rows == 0) return DSA_OK;
     if (!scores || !idx) return DSA_ERR_INVALID_ARG;
     if (ld_scores < max_len || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(scores) % 16 != 0) return DSA_ERR_INVALID_ARG;
+    if (!dsa::topk_k_supported(k)) return DSA_ERR_UNSUPPORTED_SHAPE;
     const size_t need = dsa::topk_workspace_bytes(n_rows, max_len, k);
     if (ws_bytes < need || (need > 0 && ws == nullptr)) return DSA_ERR_WORKSPACE;
     return cuda_status(dsa::launch_topk(scores, ld_scores, row_begin, n_rows, row_len, max_len, k, idx, ws,

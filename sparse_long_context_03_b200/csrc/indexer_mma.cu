@@ -138,8 +138,10 @@ __global__ void __launch_bounds__(256) indexer_prefill_mma_kernel(
     }
 }
 
+constexpr int kDecodePagesPerCta = 8;  // one page (64 keys) per warp
+
 template <int DI, int NT>
-__global__ void __launch_bounds__(256) indexer_decode_mma_kernel(
+__global__ void __launch_bounds__(256, 2) indexer_decode_mma_kernel(
     const uint8_t *__restrict__ q8, const float *__restrict__ sq, const float *__restrict__ w,
     const uint8_t *__restrict__ k8c, const float *__restrict__ skc, const int32_t *__restrict__ block_table,
     int max_pages, int num_pages, const int32_t *__restrict__ seq_lens, int max_seq_len, int HI,
@@ -148,11 +150,13 @@ __global__ void __launch_bounds__(256) indexer_decode_mma_kernel(
     const int b = blockIdx.y;
     const int n = min(min(__ldg(seq_lens + b), max_seq_len), max_pages * kPage);
     const int warp = threadIdx.x >> 5, lane = lane_id(), gid = lane >> 2, tig = lane & 3;
-    const int sb = blockIdx.x * kKeysPerCta + warp * 16;
+    const int lp = blockIdx.x * kDecodePagesPerCta + warp;   // logical page of this warp
+    const int sb = lp * kPage;
     if (sb >= n) return;
 
     // Query fragments (m16n8k32 B operand, column n = head): b0 bytes
-    // ks*32 + tig*4 of head nt*8+gid, b1 the same +16.
+    // ks*32 + tig*4 of head nt*8+gid, b1 the same +16.  Loaded once, used for
+    // the page's four 16-key tiles.
     uint32_t qf[NT][KS][2];
     float wf[NT][2];
 #pragma unroll
@@ -170,25 +174,34 @@ __global__ void __launch_bounds__(256) indexer_decode_mma_kernel(
             wf[nt][i] = hw < HI ? __ldg(w + (size_t)b * HI + hw) : 0.f;
         }
     }
-
-    const int page = __ldg(block_table + (size_t)b * max_pages + sb / kPage);
-    const bool page_ok = page >= 0 && page < num_pages;
-    const int key0 = sb + gid, key8 = key0 + 8;
-    const size_t slot0 = (size_t)(page_ok ? page : 0) * kPage + (key0 % kPage);
-    const size_t slot8 = slot0 + 8;
-    uint32_t a[KS][4];
-    load_key_frags<DI>(a, k8c + slot0 * DI, k8c + slot8 * DI, page_ok && key0 < n, page_ok && key8 < n, tig);
-    const float sk0 = (page_ok && key0 < n) ? __ldg(skc + slot0) : 0.f;
-    const float sk8 = (page_ok && key8 < n) ? __ldg(skc + slot8) : 0.f;
-
-    float p0, p1;
-    score_16keys<KS, NT>(
-        a, [&](int nt, int ks, int half) { return qf[nt][ks][half]; }, [&](int nt, int i) { return wf[nt][i]; }, p0,
-        p1);
     const float f = __ldg(sq + b);
+    const int page = __ldg(block_table + (size_t)b * max_pages + lp);
+    const bool page_ok = page >= 0 && page < num_pages;
+    const uint8_t *pk = k8c + (size_t)(page_ok ? page : 0) * kPage * DI;
+    const float *ps = skc + (size_t)(page_ok ? page : 0) * kPage;
     float *srow = scores + (size_t)b * ld;
-    if (tig == 0 && key0 < n) srow[key0] = page_ok ? p0 * f * sk0 : -INFINITY;
-    if (tig == 1 && key8 < n) srow[key8] = page_ok ? p1 * f * sk8 : -INFINITY;
+
+    // all four tiles' key fragments in flight at once
+    uint32_t a[4][KS][4];
+    float skv[4][2];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int k0 = m * 16 + gid, k8 = k0 + 8;
+        load_key_frags<DI>(a[m], pk + (size_t)k0 * DI, pk + (size_t)k8 * DI, page_ok && sb + k0 < n,
+                           page_ok && sb + k8 < n, tig);
+        skv[m][0] = (page_ok && sb + k0 < n) ? __ldg(ps + k0) : 0.f;
+        skv[m][1] = (page_ok && sb + k8 < n) ? __ldg(ps + k8) : 0.f;
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        float p0, p1;
+        score_16keys<KS, NT>(
+            a[m], [&](int nt, int ks, int half) { return qf[nt][ks][half]; },
+            [&](int nt, int i) { return wf[nt][i]; }, p0, p1);
+        const int key0 = sb + m * 16 + gid, key8 = key0 + 8;
+        if (tig == 0 && key0 < n) srow[key0] = page_ok ? p0 * f * skv[m][0] : -INFINITY;
+        if (tig == 1 && key8 < n) srow[key8] = page_ok ? p1 * f * skv[m][1] : -INFINITY;
+    }
 }
 
 // Calls launch(integral_constant<DI>, integral_constant<NT>) for a supported
@@ -240,7 +253,8 @@ cudaError_t launch_indexer_decode(const uint8_t *q8, const float *sq, const floa
                                   const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI, float *scores,
                                   int64_t ld, cudaStream_t stream) {
     if (B == 0 || max_seq_len == 0) return cudaSuccess;
-    const dim3 grid((max_seq_len + kKeysPerCta - 1) / kKeysPerCta, B);
+    const int pages = (max_seq_len + kPage - 1) / kPage;
+    const dim3 grid((pages + kDecodePagesPerCta - 1) / kDecodePagesPerCta, B);
     const bool ok = dispatch_shape(HI, dI, [&](auto di, auto nt) {
         constexpr int DI = decltype(di)::value, NT = decltype(nt)::value;
         indexer_decode_mma_kernel<DI, NT><<<grid, 256, 0, stream>>>(

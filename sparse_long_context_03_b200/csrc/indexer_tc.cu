@@ -13,14 +13,15 @@
 // owns one key and reduces over heads inside its own registers.
 //
 // Warp roles (one CTA per SM, persistent over query blocks):
-//   warp 8      TMA producer: the query block (double-buffered) and a ring
+//   warp 16     TMA producer: the query block (double-buffered) and a ring
 //               of key tiles (kStages deep);
-//   warp 9      allocates 512 TMEM columns (two 256-column accumulators) and
+//   warp 17     allocates 512 TMEM columns (two 256-column accumulators) and
 //               issues the UMMAs (dI/32 per tile), committing to mbarriers;
-//   warps 0..7  epilogue: warp w reads TMEM lanes 32*(w%4).. and columns
-//               128*(w/4).. of the finished accumulator, applies ReLU, the
-//               per-head weights (packed f32x2 FMA), the two scales and the
-//               causal mask, and stores 128 B of scores per query.
+//   warps 0..15 epilogue: warp w reads TMEM lanes 32*(w%4).. and columns
+//               64*(w/4).. of the finished accumulator (two tcgen05.ld),
+//               applies ReLU, the per-head weights (packed f32x2 FMA, four
+//               independent chains), the two scales and the causal mask, and
+//               stores 128 B of scores per query.
 // The accumulator is released as soon as its last tcgen05.ld completes, so
 // the next tile's UMMAs overlap the epilogue arithmetic.
 //
@@ -44,7 +45,10 @@ namespace {
 constexpr int kTileM = 128;     // keys per tile
 constexpr int kTileN = 256;     // (query, head) columns per tile
 constexpr int kStages = 6;      // key-tile ring depth
-constexpr int kEpiWarps = 8;
+// 4 per TMEM lane quarter, 64 columns each.  18 warps put 5 warps on two of
+// the four schedulers, whose 16K-register files then cap a thread at 96
+// registers (the launch bounds below make the compiler respect that).
+constexpr int kEpiWarps = 16;
 constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kProducerWarp = kEpiWarps;
 constexpr int kMmaWarp = kEpiWarps + 1;
@@ -78,7 +82,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const __grid_co
                                                                  int64_t ld) {
     using Lay = Layout<DI>;
     constexpr int NQ = kTileN / HI;     // queries per block
-    constexpr int QPW = NQ / 2;         // queries per epilogue warp
+    constexpr int QPW = 64 / HI;        // queries per epilogue warp (64 columns)
     constexpr int KSTEPS = DI / 32;
     constexpr uint32_t IDESC = tc::idesc_e4m3_f32(kTileM, kTileN);
 
@@ -208,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const __grid_co
     } else {
         // ------------------------------------------------------------ epilogue
         const int qw = warp & 3;        // TMEM lane quarter
-        const int half = warp >> 2;     // which 128 columns (queries half*QPW ..)
+        const int cg = warp >> 2;       // 64-column group: queries cg*QPW ..
         const uint32_t lane_base = tmem_base + ((uint32_t)(qw * 32) << 16);
         int it = 0, bi = 0;
         bool ok = true;
@@ -219,9 +223,11 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const __grid_co
             const int ntile = t_hi / kTileM + 1;
             const int wb = bi & 1;
             {   // this block's head weights and query scales into shared memory
-                const int e = threadIdx.x;  // 0..255 = (query, head)
-                const int t = t0 + e / HI;
-                w_s[wb * kTileN + e] = t <= t_hi ? __ldg(w + (size_t)t0 * HI + e) : 0.f;
+                const int e = threadIdx.x;  // 0..511; (query, head) = e for e < 256
+                if (e < kTileN) {
+                    const int t = t0 + e / HI;
+                    w_s[wb * kTileN + e] = t <= t_hi ? __ldg(w + (size_t)t0 * HI + e) : 0.f;
+                }
                 if (e < NQ) sq_s[wb * 64 + e] = (t0 + e) <= t_hi ? __ldg(sq + t0 + e) : 0.f;
                 // All epilogue warps publish before any reads (bounded wait).  A
                 // warp can only rewrite this buffer two blocks later, after every
@@ -230,44 +236,47 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const __grid_co
                 if (lane == 0) tc::mbar_arrive(wready_bar(wb));
                 if (!tc::mbar_wait(wready_bar(wb), (bi >> 1) & 1, kWaitLimitNs)) { ok = false; break; }
             }
-            const float *wq = w_s + wb * kTileN + half * QPW * HI;
+            const float *wq = w_s + wb * kTileN + cg * 64;
             for (int kt = 0; kt < ntile; ++kt, ++it) {
                 const int buf = it & 1;
-                if (!tc::mbar_wait(tfull_bar(buf), (it >> 1) & 1, kWaitLimitNs)) { ok = false; break; }
-                tc::tc_fence_after();
                 const int s = kt * kTileM + qw * 32 + lane;
                 const float sks = s <= t_hi ? __ldg(sk + s) : 0.f;
-                float2 part[QPW];
+                if (!tc::mbar_wait(tfull_bar(buf), (it >> 1) & 1, kWaitLimitNs)) { ok = false; break; }
+                tc::tc_fence_after();
+                float2 part[QPW][2];
 #pragma unroll
-                for (int q = 0; q < QPW; ++q) part[q] = make_float2(0.f, 0.f);
-                const uint32_t col0 = (uint32_t)(buf * kTileN + half * 128);
+                for (int q = 0; q < QPW; ++q) part[q][0] = part[q][1] = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 2; ++c) {
                     float acc[32];
-                    tc::tmem_ld32(lane_base + col0 + c * 32, acc);
+                    tc::tmem_ld32(lane_base + (uint32_t)(buf * kTileN + cg * 64 + c * 32), acc);
                     tc::tmem_wait_ld();
-                    if (c == 3) {  // accumulator fully read: hand it back to the MMA warp
+                    if (c == 1) {  // accumulator read: hand it back to the MMA warp before the math
                         tc::tc_fence_before();
                         __syncwarp();
                         if (lane == 0) tc::mbar_arrive(tempty_bar(buf));
                     }
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
-                        const int col = c * 32 + j;      // within this warp's 128 columns
-                        const int q = col / HI;          // compile-time after unrolling
+                        const int col = c * 32 + j;              // within this warp's 64 columns
+                        const int q = col / HI;                  // compile-time after unrolling
+                        const int chain = (j >> 2) & 1;
                         const float4 wv = *reinterpret_cast<const float4 *>(wq + col);
-                        part[q] = tc::ffma2(make_float2(wv.x, wv.y),
-                                            make_float2(fmaxf(acc[j], 0.f), fmaxf(acc[j + 1], 0.f)), part[q]);
-                        part[q] = tc::ffma2(make_float2(wv.z, wv.w),
-                                            make_float2(fmaxf(acc[j + 2], 0.f), fmaxf(acc[j + 3], 0.f)), part[q]);
+                        part[q][chain] = tc::ffma2(make_float2(wv.x, wv.y),
+                                                   make_float2(fmaxf(acc[j], 0.f), fmaxf(acc[j + 1], 0.f)),
+                                                   part[q][chain]);
+                        part[q][chain] = tc::ffma2(make_float2(wv.z, wv.w),
+                                                   make_float2(fmaxf(acc[j + 2], 0.f), fmaxf(acc[j + 3], 0.f)),
+                                                   part[q][chain]);
                     }
                 }
 #pragma unroll
                 for (int q = 0; q < QPW; ++q) {
-                    const int ql = half * QPW + q;
+                    const int ql = cg * QPW + q;
                     const int t = t0 + ql;
                     if (t <= t_hi && s <= t) {
-                        scores[(size_t)(t - row_begin) * ld + s] = (part[q].x + part[q].y) * sq_s[wb * 64 + ql] * sks;
+                        const float v = (part[q][0].x + part[q][1].x) + (part[q][0].y + part[q][1].y);
+                        scores[(size_t)(t - row_begin) * ld + s] = v * sq_s[wb * 64 + ql] * sks;
                     }
                 }
             }

@@ -26,6 +26,7 @@ cudaError_t indexer_tc_take_error(unsigned int *flag);
 
 // topk.cu
 size_t topk_workspace_bytes(int n_rows, int max_len, int k);
+bool topk_k_supported(int k);
 cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_rows, const int32_t *row_len,
                         int max_len, int k, int32_t *idx, void *ws, size_t ws_bytes, cudaStream_t stream);
 

@@ -1,24 +1,31 @@
-// topk.cu -- deterministic per-row top-k by radix select.
+// topk.cu -- deterministic per-row top-k selection.
 //
 // "Kwai Keye-VL-2.0 Technical Report" review (xllm-io), 核心公式:
 //     Omega_t = { s | I[t,s] in Top-k(I[t,:]) }
 // report translation section 5.1.2 (a row with t+1 <= k keeps all of 0..t)
 // and section 5.2.1 (the selection must be deterministic).
 //
-// Algorithm (no sort).  Scores map to order-preserving 32-bit keys (-0.0 and
-// +0.0 equal).  Three histogram passes over 11, 11 and 10 key bits find the
-// exact key T of the k-th largest score and how many entries equal to T the
-// set still needs ("quota").  A final pass walks the row in index order and
-// keeps every entry > T plus the first `quota` entries == T, writing each
-// kept index at its rank among the kept ones: the output is ascending and
-// ties go to the lower index.  Every step is a count, so the result does not
+// Scores map to order-preserving 32-bit keys (-0.0 and +0.0 equal).  The
+// selected set is every entry whose key is above the k-th largest key T,
+// plus the lowest-indexed entries equal to T; it is emitted in ascending
+// index order.  No sort, every step is a count, so the result does not
 // depend on scheduling.
 //
-// One CTA owns one row.  The first pass streams the row from HBM; later passes
-// re-read it, normally from L2 (a 128K-token row is 512 KB).  Histogram
-// increments are aggregated per warp with match.any so that the heavily
-// populated bins of the first pass (scores share sign and exponent) do not
-// serialise on one shared-memory address.
+// One CTA owns one row; three passes over the row (the first from HBM, the
+// other two normally from L2):
+//   1. the row's key range [kmin, kmax];
+//   2. a histogram over 2048 linear buckets of that range (a monotone map,
+//      so bucket order is key order; scores spread over many buckets, which
+//      keeps shared-memory atomics free of hot spots);
+//   3. an ordered collect: entries in buckets above the threshold bucket Bt
+//      are winners, written in index order to a shared list A; entries in Bt
+//      are candidates, written in index order (key, index) to a list C.
+// T is then found inside C by a small radix select in shared memory, the
+// chosen candidates are compacted (still in index order), and A and the
+// chosen candidates are merged into the output by binary search.
+// If Bt holds more candidates than fit in shared memory (massive exact ties),
+// the row falls back to a radix select over the whole row (11/11/10-bit
+// passes) followed by an ordered compaction: slower, same result.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -26,13 +33,23 @@ namespace dsa {
 
 namespace {
 
-constexpr int kTopkThreads = 512;
-constexpr int kWarps = kTopkThreads / 32;
-constexpr int kBins = 2048;
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kNB = 2048;          // linear buckets (pass 2) and radix bins
+constexpr int kCap = 6144;         // candidates kept in shared memory
+constexpr int kVec = 4;            // consecutive entries per thread per chunk
+constexpr int kChunk = kThreads * kVec;
 
-// Radix passes over the 32-bit key: bits 31..21, 20..10, 9..0.
-__device__ __forceinline__ int pass_shift(int p) { return p == 0 ? 21 : (p == 1 ? 10 : 0); }
-__device__ __forceinline__ int pass_bits(int p) { return p == 2 ? 10 : 11; }
+struct TopkSmem {
+    uint32_t hist[kNB];
+    uint32_t ckey[kCap];
+    int32_t cidx[kCap];
+    uint32_t red[2 * kWarps];
+    uint32_t bcast[4];
+    // followed by int32_t alist[k]
+};
+
+__host__ __device__ constexpr size_t smem_bytes(int k) { return sizeof(TopkSmem) + sizeof(int32_t) * (size_t)k; }
 
 __device__ __forceinline__ int row_length(const int32_t *row_len, int r, int row_begin, int max_len) {
     if (row_len == nullptr) return row_begin + r + 1;
@@ -40,12 +57,164 @@ __device__ __forceinline__ int row_length(const int32_t *row_len, int r, int row
     return n < 0 ? 0 : (n > max_len ? max_len : n);
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const float *__restrict__ scores, int64_t ld,
-                                                                int row_begin, const int32_t *__restrict__ row_len,
-                                                                int max_len, int k, int32_t *__restrict__ idx) {
-    __shared__ uint32_t hist[kBins];
-    __shared__ uint32_t warp_sum[kWarps];
-    __shared__ uint32_t sel_bin, sel_remaining;
+// Load entries i0..i0+3 (fewer at the tail) as keys; absent entries get 0.
+__device__ __forceinline__ int load4(const float *row, int i0, int n, uint32_t (&key)[kVec]) {
+    if (i0 + kVec <= n) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(row + i0));
+        key[0] = order_key(v.x);
+        key[1] = order_key(v.y);
+        key[2] = order_key(v.z);
+        key[3] = order_key(v.w);
+        return kVec;
+    }
+    int m = 0;
+#pragma unroll
+    for (int j = 0; j < kVec; ++j) {
+        key[j] = (i0 + j < n) ? order_key(__ldg(row + i0 + j)) : 0u;
+        m += (i0 + j < n);
+    }
+    return m < 0 ? 0 : m;
+}
+
+__device__ __forceinline__ uint32_t bucket_of(uint32_t key, uint32_t kmin, float scale) {
+    const uint32_t b = __float2uint_rz(__fmul_rn(__uint2float_rn(key - kmin), scale));
+    return b < (uint32_t)kNB ? b : (uint32_t)(kNB - 1);
+}
+
+// Exclusive block scan of one packed value per thread (two 16-bit counters).
+// Returns the exclusive prefix; *total gets the block total.  Two barriers.
+__device__ __forceinline__ uint32_t block_scan_packed(uint32_t v, uint32_t *red, uint32_t *total) {
+    const int lane = lane_id(), warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) red[warp] = x;
+    __syncthreads();
+    uint32_t before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        const uint32_t s = red[w];
+        before += (w < warp) ? s : 0u;
+        tot += s;
+    }
+    __syncthreads();
+    *total = tot;
+    return before + x - v;
+}
+
+// Bin b with above(b) < need <= above(b) + hist[b], above(b) = sum of bins > b;
+// thread j owns bins 4j..4j+3.  Writes (b, need - above(b), above(b)) to bcast.
+__device__ __forceinline__ void find_threshold_bin(const uint32_t *hist, uint32_t need, uint32_t *red,
+                                                   uint32_t *bcast) {
+    const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
+    uint32_t c[4], own = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        c[q] = hist[tid * 4 + q];
+        own += c[q];
+    }
+    uint32_t v = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, v, o);
+        if (lane + o < 32) v += y;
+    }
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    uint32_t above = v - own;
+    for (int w = warp + 1; w < kWarps; ++w) above += red[w];
+#pragma unroll
+    for (int q = 3; q >= 0; --q) {
+        if (above < need && need <= above + c[q]) {
+            bcast[0] = (uint32_t)(tid * 4 + q);
+            bcast[1] = need - above;
+            bcast[2] = above;
+        }
+        above += c[q];
+    }
+    __syncthreads();
+}
+
+// Radix select of the `need`-th largest key among ckey[0..cnt): returns T and
+// how many entries equal to T are to be taken.
+__device__ __forceinline__ void select_in_candidates(TopkSmem &sm, int cnt, uint32_t need, uint32_t &T,
+                                                     uint32_t &quota) {
+    uint32_t prefix = 0, pmask = 0;
+#pragma unroll 1
+    for (int p = 0; p < 3; ++p) {
+        const int shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
+        const uint32_t dmask = (p == 2 ? 1023u : 2047u);
+        for (int i = threadIdx.x; i < kNB; i += kThreads) sm.hist[i] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < cnt; i += kThreads) {
+            const uint32_t key = sm.ckey[i];
+            if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & dmask], 1u);
+        }
+        __syncthreads();
+        find_threshold_bin(sm.hist, need, sm.red, sm.bcast);
+        prefix |= sm.bcast[0] << shift;
+        pmask |= dmask << shift;
+        need = sm.bcast[1];
+        __syncthreads();
+    }
+    T = prefix;
+    quota = need;
+}
+
+// Slow exact path over the whole row (used when the threshold bucket does
+// not fit in shared memory): radix select then ordered compaction.
+__device__ void topk_row_radix(const float *row, int n, int k, int32_t *out, TopkSmem &sm) {
+    const int tid = threadIdx.x, lane = lane_id();
+    uint32_t prefix = 0, pmask = 0, need = (uint32_t)k;
+#pragma unroll 1
+    for (int p = 0; p < 3; ++p) {
+        const int shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
+        const uint32_t dmask = (p == 2 ? 1023u : 2047u);
+        for (int i = tid; i < kNB; i += kThreads) sm.hist[i] = 0;
+        __syncthreads();
+        for (int base = (tid >> 5) * 32; base < n; base += kThreads) {
+            const int i = base + lane;
+            uint32_t bin = 0xFFFFFFFFu;
+            if (i < n) {
+                const uint32_t key = order_key(__ldg(row + i));
+                if ((key & pmask) == prefix) bin = (key >> shift) & dmask;
+            }
+            const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+            if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], __popc(peers));
+        }
+        __syncthreads();
+        find_threshold_bin(sm.hist, need, sm.red, sm.bcast);
+        prefix |= sm.bcast[0] << shift;
+        pmask |= dmask << shift;
+        need = sm.bcast[1];
+        __syncthreads();
+    }
+    const uint32_t T = prefix, quota = need;
+    uint32_t run_gt = 0, run_eq = 0;
+    for (int base = 0; base < n; base += kThreads) {
+        const int i = base + tid;
+        const uint32_t key = i < n ? order_key(__ldg(row + i)) : 0u;
+        const bool gt = i < n && key > T;
+        const bool eq = i < n && key == T;
+        uint32_t tot;
+        const uint32_t ex = block_scan_packed((gt ? 1u : 0u) | (eq ? 0x10000u : 0u), sm.red, &tot);
+        const uint32_t gt_before = run_gt + (ex & 0xFFFFu);
+        const uint32_t eq_before = run_eq + (ex >> 16);
+        if (gt || (eq && eq_before < quota)) out[gt_before + min(eq_before, quota)] = i;
+        run_gt += tot & 0xFFFFu;
+        run_eq += tot >> 16;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__restrict__ scores, int64_t ld,
+                                                            int row_begin, const int32_t *__restrict__ row_len,
+                                                            int max_len, int k, int32_t *__restrict__ idx) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    int32_t *alist = reinterpret_cast<int32_t *>(smem_raw + sizeof(TopkSmem));
 
     const int r = blockIdx.x;
     const int n = row_length(row_len, r, row_begin, max_len);
@@ -54,92 +223,137 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const float *__
     const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
 
     if (n <= k) {  // short row: everything visible is selected
-        for (int i = tid; i < k; i += kTopkThreads) out[i] = i < n ? i : -1;
+        for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
         return;
     }
 
-    uint32_t prefix = 0, pmask = 0;
-    uint32_t remaining = (uint32_t)k;
-#pragma unroll 1
-    for (int p = 0; p < 3; ++p) {
-        const int shift = pass_shift(p);
-        const uint32_t dmask = (1u << pass_bits(p)) - 1u;
-        for (int i = tid; i < kBins; i += kTopkThreads) hist[i] = 0;
-        __syncthreads();
-        for (int base = warp * 32; base < n; base += kTopkThreads) {
-            const int i = base + lane;
-            uint32_t bin = 0xFFFFFFFFu;
-            if (i < n) {
-                const uint32_t key = order_key(row[i]);
-                if ((key & pmask) == prefix) bin = (key >> shift) & dmask;
+    // ---- pass 1: key range
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int i0 = tid * kVec; i0 < n; i0 += kChunk) {
+        uint32_t key[kVec];
+        const int m = load4(row, i0, n, key);
+#pragma unroll
+        for (int j = 0; j < kVec; ++j) {
+            if (j < m) {
+                kmin = min(kmin, key[j]);
+                kmax = max(kmax, key[j]);
             }
-            const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
-            if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
         }
-        __syncthreads();
+    }
+    kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
+    kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+    if (lane == 0) {
+        sm.red[warp] = kmin;
+        sm.red[kWarps + warp] = kmax;
+    }
+    for (int i = tid; i < kNB; i += kThreads) sm.hist[i] = 0;
+    __syncthreads();
+    kmin = sm.red[0];
+    kmax = sm.red[kWarps];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) {
+        kmin = min(kmin, sm.red[w]);
+        kmax = max(kmax, sm.red[kWarps + w]);
+    }
+    if (kmin == kmax) {  // every entry ties: the k lowest indices
+        for (int i = tid; i < k; i += kThreads) out[i] = i;
+        return;
+    }
+    const float scale = (float)kNB / ((float)(kmax - kmin) + 1.0f);
 
-        // Bin b holds the k-th largest iff above(b) < remaining <= above(b) + hist[b],
-        // above(b) = sum of bins > b.  Thread j owns bins 4j..4j+3; a block
-        // suffix sum over threads gives each thread the count above its bins.
-        uint32_t c[4], own = 0;
+    // ---- pass 2: bucket histogram
+    for (int i0 = tid * kVec; i0 < n; i0 += kChunk) {
+        uint32_t key[kVec];
+        const int m = load4(row, i0, n, key);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            c[q] = hist[tid * 4 + q];
-            own += c[q];
+        for (int j = 0; j < kVec; ++j)
+            if (j < m) atomicAdd(&sm.hist[bucket_of(key[j], kmin, scale)], 1u);
+    }
+    __syncthreads();
+    find_threshold_bin(sm.hist, (uint32_t)k, sm.red, sm.bcast);
+    const uint32_t Bt = sm.bcast[0];
+    const uint32_t need = sm.bcast[1];       // taken from the threshold bucket
+    const uint32_t n_above = sm.bcast[2];    // entries in buckets above it
+    const uint32_t cnt = sm.hist[Bt];
+    __syncthreads();
+
+    if (cnt > (uint32_t)kCap) {
+        topk_row_radix(row, n, k, out, sm);
+        return;
+    }
+
+    // ---- pass 3: ordered collect
+    uint32_t run_a = 0, run_c = 0;
+    for (int base = 0; base < n; base += kChunk) {
+        const int i0 = base + tid * kVec;
+        uint32_t key[kVec] = {0u, 0u, 0u, 0u};
+        const int m = i0 < n ? load4(row, i0, n, key) : 0;
+        uint32_t cls[kVec];
+        uint32_t na = 0, nc = 0;
+#pragma unroll
+        for (int j = 0; j < kVec; ++j) {
+            const uint32_t b = bucket_of(key[j], kmin, scale);
+            cls[j] = j >= m ? 0u : (b > Bt ? 2u : (b == Bt ? 1u : 0u));
+            na += cls[j] == 2u;
+            nc += cls[j] == 1u;
         }
-        // inclusive scan from the top: thread order reversed
-        uint32_t v = own;
+        uint32_t tot;
+        const uint32_t ex = block_scan_packed(na | (nc << 16), sm.red, &tot);
+        uint32_t pa = run_a + (ex & 0xFFFFu), pc = run_c + (ex >> 16);
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, v, o);
-            if (lane + o < 32) v += y;
-        }
-        if (lane == 0) warp_sum[warp] = v;  // total of this warp
-        __syncthreads();
-        uint32_t above = v - own;  // bins owned by higher lanes of this warp
-        for (int w2 = warp + 1; w2 < kWarps; ++w2) above += warp_sum[w2];
-#pragma unroll
-        for (int q = 3; q >= 0; --q) {
-            if (above < remaining && remaining <= above + c[q]) {
-                sel_bin = (uint32_t)(tid * 4 + q);
-                sel_remaining = remaining - above;
+        for (int j = 0; j < kVec; ++j) {
+            if (cls[j] == 2u) alist[pa++] = i0 + j;
+            if (cls[j] == 1u) {
+                sm.ckey[pc] = key[j];
+                sm.cidx[pc] = i0 + j;
+                ++pc;
             }
-            above += c[q];
         }
-        __syncthreads();
-        prefix |= sel_bin << shift;
-        pmask |= dmask << shift;
-        remaining = sel_remaining;
+        run_a += tot & 0xFFFFu;
+        run_c += tot >> 16;
+    }
+    __syncthreads();
+
+    // ---- threshold key inside the candidates, then keep the chosen ones
+    uint32_t T, quota;
+    select_in_candidates(sm, (int)cnt, need, T, quota);
+    uint32_t run_g = 0, run_e = 0;
+    for (int base = 0; base < (int)cnt; base += kThreads) {
+        const int i = base + tid;
+        const uint32_t key = i < (int)cnt ? sm.ckey[i] : 0u;
+        const int32_t ix = i < (int)cnt ? sm.cidx[i] : 0;
+        const bool gt = i < (int)cnt && key > T;
+        const bool eq = i < (int)cnt && key == T;
+        uint32_t tot;
+        const uint32_t ex = block_scan_packed((gt ? 1u : 0u) | (eq ? 0x10000u : 0u), sm.red, &tot);
+        const uint32_t gb = run_g + (ex & 0xFFFFu), eb = run_e + (ex >> 16);
+        // positions only move left and this chunk was read before the scan's barriers
+        if (gt || (eq && eb < quota)) sm.cidx[gb + min(eb, quota)] = ix;
+        run_g += tot & 0xFFFFu;
+        run_e += tot >> 16;
         __syncthreads();
     }
 
-    // Ordered compaction: keep key > T, and key == T while the quota lasts.
-    const uint32_t T = prefix;
-    const uint32_t quota = remaining;
-    const uint32_t lt = (1u << lane) - 1u;
-    uint32_t run_gt = 0, run_eq = 0;
-    for (int base = 0; base < n; base += kTopkThreads) {
-        const int i = base + tid;
-        uint32_t key = 0;
-        if (i < n) key = order_key(row[i]);
-        const bool gt = i < n && key > T;
-        const bool eq = i < n && key == T;
-        const uint32_t bg = __ballot_sync(0xFFFFFFFFu, gt), be = __ballot_sync(0xFFFFFFFFu, eq);
-        if (lane == 0) warp_sum[warp] = __popc(bg) | (__popc(be) << 16);
-        __syncthreads();
-        uint32_t before = 0, total = 0;
-#pragma unroll
-        for (int w2 = 0; w2 < kWarps; ++w2) {
-            const uint32_t x = warp_sum[w2];
-            before += (w2 < warp) ? x : 0u;
-            total += x;
+    // ---- merge the two ascending lists into the output
+    const int na = (int)n_above, nd = (int)need;
+    const int32_t *dl = sm.cidx;
+    for (int a = tid; a < na; a += kThreads) {
+        const int32_t v = alist[a];
+        int lo = 0, hi = nd;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (dl[mid] < v) lo = mid + 1; else hi = mid;
         }
-        const uint32_t gt_before = run_gt + (before & 0xFFFFu) + __popc(bg & lt);
-        const uint32_t eq_before = run_eq + (before >> 16) + __popc(be & lt);
-        if (gt || (eq && eq_before < quota)) out[gt_before + min(eq_before, quota)] = i;
-        run_gt += total & 0xFFFFu;
-        run_eq += total >> 16;
-        __syncthreads();
+        out[a + lo] = v;
+    }
+    for (int d = tid; d < nd; d += kThreads) {
+        const int32_t v = dl[d];
+        int lo = 0, hi = na;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (alist[mid] < v) lo = mid + 1; else hi = mid;
+        }
+        out[d + lo] = v;
     }
 }
 
@@ -150,8 +364,14 @@ size_t topk_workspace_bytes(int, int, int) { return 0; }
 cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_rows, const int32_t *row_len,
                         int max_len, int k, int32_t *idx, void *, size_t, cudaStream_t stream) {
     if (n_rows == 0) return cudaSuccess;
-    topk_rows_kernel<<<n_rows, kTopkThreads, 0, stream>>>(scores, ld, row_begin, row_len, max_len, k, idx);
+    const size_t smem = smem_bytes(k);
+    if (smem > 220 * 1024) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    topk_rows_kernel<<<n_rows, kThreads, smem, stream>>>(scores, ld, row_begin, row_len, max_len, k, idx);
     return cudaGetLastError();
 }
+
+bool topk_k_supported(int k) { return smem_bytes(k) <= 220 * 1024; }
 
 }  // namespace dsa

@@ -122,6 +122,31 @@ def test_topk_chunk_offset_and_determinism():
     assert np.array_equal(a, ref)
 
 
+def test_topk_fallback_massive_ties():
+    # Three distinct values over 100000 entries: the threshold bucket holds
+    # ~33K entries, more than shared memory stages, so the whole-row radix
+    # path decides; the result must be the same deterministic set.
+    rng = np.random.default_rng(3)
+    x = rng.choice(np.array([0.5, 1.0, 2.0], np.float32), size=(3, 100000))
+    x[2, :] = 1.0
+    x[2, 77777] = 3.0
+    got = gpu_topk(x, 2048, row_len=[100000, 99999, 100000])
+    ref = oracle.topk(x.astype(np.float64), [100000, 99999, 100000], 2048)
+    assert np.array_equal(got, ref)
+
+
+def test_topk_clustered_near_ties():
+    # Frame-like clusters: groups of 256 scores within 1e-6 relative of each
+    # other, as the multimodal workload produces.
+    rng = np.random.default_rng(11)
+    n = 50000
+    centers = rng.standard_normal(n // 256 + 1).astype(np.float32)
+    x = (np.repeat(centers, 256)[:n] * (1 + 1e-6 * rng.standard_normal(n))).astype(np.float32)[None, :]
+    for k in (64, 2048, 2047):
+        got = gpu_topk(x, k, row_len=[n])
+        assert np.array_equal(got, oracle.topk(x.astype(np.float64), [n], k))
+
+
 def test_topk_signed_zeros_and_all_equal():
     x = np.zeros((3, 100), np.float32)
     x[0, ::2] = -0.0
