@@ -204,6 +204,37 @@ DSA_API dsa_status_t dsa_sparse_gqa_decode_attention(const uint16_t *q,
                                              void *ws, size_t ws_bytes,
                                              uint16_t *out, float *lse, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Decode attention that allocates nothing.
+ *
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory themselves: a plugin or serving hook that is
+ * handed only its input and output buffers, or a latency-critical loop in
+ * which cudaMalloc (which may synchronise the device, and may fail under
+ * memory pressure) is not allowed.  It computes exactly what
+ * dsa_sparse_gqa_decode_attention computes, with the same arguments minus the
+ * workspace: the split-K partials live in a fixed array inside the library
+ * (dsa_decode_attention_fixed_scratch_bytes() bytes, 8 MiB), which every GPU
+ * that loads the library holds until the process exits.
+ *  - Limit: B * Hkv * 8 * (D + 2) * 4 bytes must fit that array (B <= 504
+ *    for Hkv = 4, D = 128); larger batches return DSA_ERR_WORKSPACE without
+ *    launching.  Within the limit the split count may be lower than the
+ *    workspace variant's, so results can differ from it by rounding only.
+ *  - The first call on a device looks up the array's device address with
+ *    that device current; make that first call before any stream capture.
+ *  - Every call on a device shares the one array: calls whose executions
+ *    overlap on the GPU (other streams, other host threads) race.  Nothing
+ *    has to be cleared between calls; each call writes every partial it reads.
+ *  - No cudaMalloc, cudaFree or allocating library routine is called.
+ * ------------------------------------------------------------------------ */
+DSA_API size_t dsa_decode_attention_fixed_scratch_bytes(void);
+DSA_API dsa_status_t dsa_sparse_gqa_decode_attention_noalloc(const uint16_t *q,
+                                             const uint16_t *k_cache, const uint16_t *v_cache,
+                                             const int32_t *block_table, int max_pages, int num_pages,
+                                             const int32_t *seq_lens, const int32_t *idx,
+                                             int B, int Hq, int Hkv, int D, int k, float sm_scale,
+                                             uint16_t *out, float *lse, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

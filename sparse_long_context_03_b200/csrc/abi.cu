@@ -158,6 +158,30 @@ dsa_status_t dsa_sparse_gqa_decode_attention(const uint16_t *q, const uint16_t *
                                                  as_stream(stream)));
 }
 
+size_t dsa_decode_attention_fixed_scratch_bytes(void) { return dsa::fixed_scratch_bytes(); }
+
+dsa_status_t dsa_sparse_gqa_decode_attention_noalloc(const uint16_t *q, const uint16_t *k_cache,
+                                                     const uint16_t *v_cache, const int32_t *block_table,
+                                                     int max_pages, int num_pages, const int32_t *seq_lens,
+                                                     const int32_t *idx, int B, int Hq, int Hkv, int D, int k,
+                                                     float sm_scale, uint16_t *out, float *lse, void *stream) {
+    if (B < 0 || k < 1 || Hq < 1 || Hkv < 1 || max_pages < 1 || num_pages < 1) return DSA_ERR_INVALID_ARG;
+    if (!dsa::attention_shape_supported(Hq, Hkv, D)) return DSA_ERR_UNSUPPORTED_SHAPE;
+    if (B == 0) return DSA_OK;
+    if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !idx || !out) return DSA_ERR_INVALID_ARG;
+    if (dsa::fixed_scratch_max_split(B, Hkv, D) < 1) {
+        std::strncpy(g_last_error,
+                     "batch too large for the fixed decode scratch: B * Hkv * 8 * (D + 2) * 4 bytes must not "
+                     "exceed dsa_decode_attention_fixed_scratch_bytes()",
+                     sizeof(g_last_error) - 1);
+        g_last_error[sizeof(g_last_error) - 1] = '\0';
+        return DSA_ERR_WORKSPACE;
+    }
+    return cuda_status(dsa::launch_sparse_decode_fixed_scratch(q, k_cache, v_cache, block_table, max_pages,
+                                                               num_pages, seq_lens, idx, B, Hq, Hkv, D, k, sm_scale,
+                                                               out, lse, as_stream(stream)));
+}
+
 size_t dsa_decode_workspace_size(int B, int max_seq_len, int Hq, int Hkv, int D, int k) {
     if (B < 0 || max_seq_len < 0 || Hkv < 1 || k < 1 || D < 1) return 0;
     return decode_ws_layout(B, max_seq_len, Hq, Hkv, D, k).total;

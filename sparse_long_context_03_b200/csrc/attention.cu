@@ -24,6 +24,7 @@
 // Decode: the k selected rows of a (sequence, group) are split across warps
 // (split-K); each split writes (max, sum, unnormalised O) to the workspace and
 // a combine kernel merges them.
+#include <atomic>
 #include <type_traits>
 
 #include "common.cuh"
@@ -416,6 +417,105 @@ cudaError_t launch_sparse_decode(const uint16_t *q, const uint16_t *k_cache, con
     const int grid = (items + kWarpsPerCta - 1) / kWarpsPerCta;
     float *part = static_cast<float *>(ws);
     cudaError_t err = cudaSuccess;
+    const bool ok = dispatch_d(D, [&](auto dc) {
+        constexpr int DD = decltype(dc)::value;
+        constexpr int smem = kWarpsPerCta * warp_smem_bytes<DD>();
+        err = cudaFuncSetAttribute(sparse_decode_split_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   smem);
+        if (err != cudaSuccess) return true;
+        sparse_decode_split_kernel<DD><<<grid, kWarpsPerCta * 32, smem, stream>>>(
+            q, k_cache, v_cache, block_table, max_pages, num_pages, seq_lens, idx, B, Hq, Hkv, k, s.chunk, s.nsplit,
+            sm_scale * kLog2e, part);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return true;
+        decode_combine_kernel<DD><<<B * Hq, DD, 0, stream>>>(part, Hq, Hkv, s.nsplit, out, lse);
+        err = cudaGetLastError();
+        return true;
+    });
+    return ok ? err : cudaErrorInvalidValue;
+}
+
+}  // namespace dsa
+
+// ---------------------------------------------------------------------------
+// Decode attention for callers that cannot allocate device memory.
+//
+// The split-K partials of the decode attention normally live in a workspace
+// the caller allocates.  This variant keeps them in a fixed array that is part
+// of the library image instead: every GPU that loads the library holds
+// kFixedScratchBytes of it until the process exits.  All calls on a device
+// share the array, so calls whose executions overlap on that device race.
+// Every partial the combine pass reads is written by the split pass of the
+// same call, so nothing has to be cleared between calls.
+// ---------------------------------------------------------------------------
+
+namespace dsa {
+constexpr size_t kFixedScratchBytes = size_t(8) << 20;  // 8 MiB
+}  // namespace dsa
+
+static __device__ __align__(256) float g_decode_fixed_scratch[dsa::kFixedScratchBytes / sizeof(float)];
+
+namespace dsa {
+
+namespace {
+
+// Device address of g_decode_fixed_scratch on the current device.  In host
+// code the array's name is only a host-side stand-in, so the address is
+// looked up once per device (with that device current) and cached.
+float *fixed_scratch_on_current_device(cudaError_t *err) {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<float *> cached[kMaxDevices];
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess) return nullptr;
+    if (dev < 0 || dev >= kMaxDevices) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    float *p = cached[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+        void *addr = nullptr;
+        *err = cudaGetSymbolAddress(&addr, g_decode_fixed_scratch);
+        if (*err != cudaSuccess) return nullptr;
+        p = static_cast<float *>(addr);
+        cached[dev].store(p, std::memory_order_release);
+    }
+    return p;
+}
+
+}  // namespace
+
+size_t fixed_scratch_bytes() { return kFixedScratchBytes; }
+
+// Largest split count whose partials fit the fixed array (0 if even one split
+// does not fit).
+int fixed_scratch_max_split(int B, int Hkv, int D) {
+    const size_t per_split = (size_t)B * Hkv * 8 * (D + 2) * sizeof(float);
+    if (per_split == 0) return 1 << 30;
+    const size_t n = kFixedScratchBytes / per_split;
+    return n > (size_t)(1 << 30) ? (1 << 30) : (int)n;
+}
+
+cudaError_t launch_sparse_decode_fixed_scratch(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                                               const int32_t *block_table, int max_pages, int num_pages,
+                                               const int32_t *seq_lens, const int32_t *idx, int B, int Hq, int Hkv,
+                                               int D, int k, float sm_scale, uint16_t *out, float *lse,
+                                               cudaStream_t stream) {
+    if (B == 0) return cudaSuccess;
+    const int cap = fixed_scratch_max_split(B, Hkv, D);
+    if (cap < 1) return cudaErrorInvalidValue;
+    cudaError_t err = cudaSuccess;
+    float *part = fixed_scratch_on_current_device(&err);
+    if (part == nullptr) return err;
+    // Same split rule as the workspace variant, capped so the partials fit.
+    DecodeSplit s = decode_split(B, Hkv, k);
+    if (s.nsplit > cap) {
+        int chunk = (k + cap - 1) / cap;
+        chunk = (chunk + kBlk - 1) / kBlk * kBlk;
+        s = {chunk, (k + chunk - 1) / chunk};
+    }
+    const int items = B * Hkv * s.nsplit;
+    const int grid = (items + kWarpsPerCta - 1) / kWarpsPerCta;
     const bool ok = dispatch_d(D, [&](auto dc) {
         constexpr int DD = decltype(dc)::value;
         constexpr int smem = kWarpsPerCta * warp_smem_bytes<DD>();

@@ -41,4 +41,14 @@ cudaError_t launch_sparse_decode(const uint16_t *q, const uint16_t *k_cache, con
                                  const int32_t *idx, int B, int Hq, int Hkv, int D, int k, float sm_scale,
                                  void *ws, size_t ws_bytes, uint16_t *out, float *lse, cudaStream_t stream);
 
+// attention.cu: decode attention with its split-K partials in a fixed device
+// array of the library (for callers that cannot allocate)
+size_t fixed_scratch_bytes();
+int fixed_scratch_max_split(int B, int Hkv, int D);
+cudaError_t launch_sparse_decode_fixed_scratch(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                                               const int32_t *block_table, int max_pages, int num_pages,
+                                               const int32_t *seq_lens, const int32_t *idx, int B, int Hq, int Hkv,
+                                               int D, int k, float sm_scale, uint16_t *out, float *lse,
+                                               cudaStream_t stream);
+
 }  // namespace dsa

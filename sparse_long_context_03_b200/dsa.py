@@ -44,6 +44,9 @@ _SIGNATURES = {
     "dsa_decode_attention_workspace_size": ([_I, _I, _I, _I, _I], _SZ),
     "dsa_sparse_gqa_decode_attention": ([_P, _P, _P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _I, _F,
                                          _P, _SZ, _P, _P, _P], _I),
+    "dsa_decode_attention_fixed_scratch_bytes": ([], _SZ),
+    "dsa_sparse_gqa_decode_attention_noalloc": ([_P, _P, _P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _I, _F,
+                                                 _P, _P, _P], _I),
 }
 
 
@@ -251,3 +254,26 @@ def sparse_gqa_decode(q, q8, q_scale, w, k8_cache, k_scale_cache, k_cache, v_cac
                                        Hq, Hkv, D, HI, dI, int(k), float(sm_scale), _ptr(ws),
                                        ws.numel() * ws.element_size(), _ptr(out), _ptr(idx_out), _stream(stream)),
            "dsa_sparse_gqa_decode")
+
+
+def decode_attention_fixed_scratch_bytes() -> int:
+    return int(lib().dsa_decode_attention_fixed_scratch_bytes())
+
+
+def sparse_gqa_decode_attention_noalloc(q, k_cache, v_cache, block_table, seq_lens, idx, k, sm_scale, out, lse=None,
+                                        stream=None):
+    """dsa_sparse_gqa_decode_attention_noalloc: the decode attention with no
+    caller workspace (its scratch is a fixed array inside the library).  For
+    callers that cannot allocate device memory; calls that overlap on one
+    GPU race on that array."""
+    _need(q, torch.bfloat16, 3, "q")
+    _need(k_cache, torch.bfloat16, 4, "k_cache")
+    _need(v_cache, torch.bfloat16, 4, "v_cache")
+    _need(out, torch.bfloat16, 3, "out")
+    B, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    _check(lib().dsa_sparse_gqa_decode_attention_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                                         block_table.shape[1], k_cache.shape[0], _ptr(seq_lens),
+                                                         _ptr(idx), B, Hq, Hkv, D, int(k), float(sm_scale),
+                                                         _ptr(out), _ptr(lse), _stream(stream)),
+           "dsa_sparse_gqa_decode_attention_noalloc")
