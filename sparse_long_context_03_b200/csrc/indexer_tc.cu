@@ -8,22 +8,24 @@
 //     I[t,s] = sq[t] * sk[s] * sum_j w[t,j] * ReLU(q8[t,j] . k8[s]).
 //
 // GEMM view: A = 128 keys x dI (K-major, TMA tile), B = NQ queries x HI heads
-// = 256 rows x dI (K-major, one query block), D = 128 x 256 fp32 in TMEM
+// = 128 rows x dI (K-major, one query block), D = 128 x 128 fp32 in TMEM
 // (lane = key, column = (query, head)).  Keys on M means one epilogue thread
 // owns one key and reduces over heads inside its own registers.
 //
 // Warp roles (one CTA per SM, persistent over query blocks):
-//   warp 16     TMA producer: the query block (double-buffered) and a ring
-//               of key tiles (kStages deep);
-//   warp 17     allocates 512 TMEM columns (two 256-column accumulators) and
-//               issues the UMMAs (dI/32 per tile), committing to mbarriers;
-//   warps 0..15 epilogue: warp w reads TMEM lanes 32*(w%4).. and columns
-//               64*(w/4).. of the finished accumulator (two tcgen05.ld),
-//               applies ReLU, the per-head weights (packed f32x2 FMA, four
-//               independent chains), the two scales and the causal mask, and
-//               stores 128 B of scores per query.
-// The accumulator is released as soon as its last tcgen05.ld completes, so
-// the next tile's UMMAs overlap the epilogue arithmetic.
+//   producer    TMA: the query block (double-buffered) and a ring of key
+//               tiles (kStages deep);
+//   MMA         allocates 512 TMEM columns (four 128-column accumulators)
+//               and issues the UMMAs (dI/32 per tile), committing to
+//               mbarriers;
+//   epilogue    4 x (128 / CW) warps: warp w reads TMEM lanes 32*(w%4).. and
+//               the CW = max(32, HI) columns of one query (or 32/HI whole
+//               queries) with 32x32b loads, so each thread holds one key and
+//               its query's head weights live in registers for the whole
+//               query block: ReLU, weighted head sum (packed f32x2 FMA), the
+//               two scales and the causal mask, then a coalesced store.
+// An accumulator is handed back as soon as its last tcgen05.ld completes; with
+// four of them the UMMAs run up to three tiles ahead of the epilogue.
 //
 // Every mbarrier wait is bounded (globaltimer); on timeout the kernel sets
 // an error flag, every role unwinds, and TMEM is freed before exit.
@@ -42,29 +44,44 @@ __device__ unsigned int g_indexer_tc_error;
 
 namespace {
 
-constexpr int kTileM = 128;     // keys per tile
-constexpr int kTileN = 256;     // (query, head) columns per tile
-constexpr int kStages = 6;      // key-tile ring depth
-// 4 per TMEM lane quarter, 64 columns each.  18 warps put 5 warps on two of
-// the four schedulers, whose 16K-register files then cap a thread at 96
-// registers (the launch bounds below make the compiler respect that).
-constexpr int kEpiWarps = 16;
-constexpr int kThreads = (kEpiWarps + 2) * 32;
-constexpr int kProducerWarp = kEpiWarps;
-constexpr int kMmaWarp = kEpiWarps + 1;
+constexpr int kTileM = 128;     // keys per MMA (UMMA M)
+constexpr int kTileN = 128;     // (query, head) columns per tile
+constexpr int kStepKeys = 256;  // keys per pipeline step: two MMA tiles
+constexpr int kAccBufs = 4;     // TMEM accumulators (4 x 128 = 512 columns) ...
+constexpr int kPairs = kAccBufs / 2;  // ... used in pairs, one pair per step
 constexpr uint32_t kTmemCols = 512;
+
+// With dI = 64 a tile needs only two MMAs, so the single MMA thread's fixed
+// cost per step (barrier waits, fences, commits) sets the pace; a step of two
+// tiles (one 256-row TMA box, 2 x dI/32 MMAs into an accumulator pair, one
+// commit) halves that cost per MMA.
+
+// Columns per epilogue warp and the warp counts for HI heads per query.  With
+// 18 warps, two of the four schedulers hold five warps, whose 16K-register
+// files cap a thread at 96 registers (HI <= 32); HI = 64 has 10 warps.
+template <int HI>
+struct EpiShape {
+    static constexpr int CW = HI > 32 ? HI : 32;
+    static constexpr int kEpiWarps = 4 * (kTileN / CW);
+    static constexpr int kThreads = (kEpiWarps + 2) * 32;
+    static constexpr int kProducerWarp = kEpiWarps;
+    static constexpr int kMmaWarp = kEpiWarps + 1;
+};
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+constexpr uint32_t kIssuerSleepNs = 32;            // back-off of the TMA and MMA warps
+
 
 template <int DI>
 struct Layout {
-    static constexpr int kTileBytes = kTileM * DI;
+    static constexpr int kTileBytes = kStepKeys * DI;  // one step of keys
+    static constexpr int kStages = (200 * 1024 - 2 * kTileN * DI) / kTileBytes > 8
+                                       ? 8
+                                       : (200 * 1024 - 2 * kTileN * DI) / kTileBytes;
     static constexpr int kQBytes = kTileN * DI;
     static constexpr int kKeys = 0;
     static constexpr int kQ = kKeys + kStages * kTileBytes;
-    static constexpr int kW = kQ + 2 * kQBytes;                  // float [2][256]
-    static constexpr int kSq = kW + 2 * kTileN * 4;             // float [2][64]
-    static constexpr int kBars = kSq + 2 * 64 * 4;              // uint64 barriers
-    static constexpr int kNumBars = 2 * kStages + 11;
+    static constexpr int kBars = kQ + 2 * kQBytes;              // uint64 barriers
+    static constexpr int kNumBars = 2 * kStages + 4 + 2 * kPairs + 1;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kBytes = kTmemSlot + 16;
     static constexpr int kAlloc = kBytes + 1024;                // slack for 1024-byte alignment
@@ -73,7 +90,7 @@ struct Layout {
 __device__ __forceinline__ void record_timeout() { atomicOr(&g_indexer_tc_error, 1u); }
 
 template <int HI, int DI>
-__global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
+__global__ void __launch_bounds__(EpiShape<HI>::kThreads, 1) indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                                                  const __grid_constant__ CUtensorMap tmap_q,
                                                                  const float *__restrict__ sq,
                                                                  const float *__restrict__ w,
@@ -81,25 +98,26 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const __grid_co
                                                                  int n_rows, float *__restrict__ scores,
                                                                  int64_t ld) {
     using Lay = Layout<DI>;
+    using ES = EpiShape<HI>;
+    constexpr int kEpiWarps = ES::kEpiWarps, kProducerWarp = ES::kProducerWarp, kMmaWarp = ES::kMmaWarp;
+    constexpr int CW = ES::CW;          // columns per epilogue warp
     constexpr int NQ = kTileN / HI;     // queries per block
-    constexpr int QPW = 64 / HI;        // queries per epilogue warp (64 columns)
+    constexpr int QPW = CW / HI;        // whole queries per epilogue warp (1 when HI >= 32)
     constexpr int KSTEPS = DI / 32;
+    constexpr int kStages = Lay::kStages;
     constexpr uint32_t IDESC = tc::idesc_e4m3_f32(kTileM, kTileN);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    float *w_s = reinterpret_cast<float *>(smem + Lay::kW);
-    float *sq_s = reinterpret_cast<float *>(smem + Lay::kSq);
     const uint32_t bars = sbase + Lay::kBars;
     auto full_bar = [&](int s) { return bars + 8u * s; };
     auto empty_bar = [&](int s) { return bars + 8u * (kStages + s); };
     auto qfull_bar = [&](int b) { return bars + 8u * (2 * kStages + b); };
     auto qempty_bar = [&](int b) { return bars + 8u * (2 * kStages + 2 + b); };
     auto tfull_bar = [&](int b) { return bars + 8u * (2 * kStages + 4 + b); };
-    auto tempty_bar = [&](int b) { return bars + 8u * (2 * kStages + 6 + b); };
-    auto wready_bar = [&](int b) { return bars + 8u * (2 * kStages + 8 + b); };
-    const uint32_t mma_done_bar = bars + 8u * (2 * kStages + 10);
+    auto tempty_bar = [&](int b) { return bars + 8u * (2 * kStages + 4 + kPairs + b); };
+    const uint32_t mma_done_bar = bars + 8u * (2 * kStages + 4 + 2 * kPairs);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + Lay::kTmemSlot);
 
     const int warp = threadIdx.x >> 5, lane = lane_id();
@@ -114,9 +132,10 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const __grid_co
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(qfull_bar(b), 1);
             tc::mbar_init(qempty_bar(b), 1);
+        }
+        for (int b = 0; b < kPairs; ++b) {
             tc::mbar_init(tfull_bar(b), 1);
             tc::mbar_init(tempty_bar(b), kEpiWarps);
-            tc::mbar_init(wready_bar(b), kEpiWarps);
         }
         tc::mbar_init(mma_done_bar, 1);
         tc::fence_mbar_init();
@@ -145,16 +164,22 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const __grid_co
                 const int qb = nb - 1 - i;
                 const int t0 = row_begin + qb * NQ;
                 const int t_hi = min(t0 + NQ, row_end) - 1;
-                const int ntile = t_hi / kTileM + 1;
+                const int nstep = t_hi / kStepKeys + 1;
                 const int qs = bi & 1;
-                if (!tc::mbar_wait(qempty_bar(qs), ((bi >> 1) & 1) ^ 1, kWaitLimitNs)) { ok = false; break; }
+                if (!tc::mbar_wait_sleep(qempty_bar(qs), ((bi >> 1) & 1) ^ 1, kWaitLimitNs, kIssuerSleepNs)) {
+                    ok = false;
+                    break;
+                }
                 tc::mbar_arrive_expect_tx(qfull_bar(qs), Lay::kQBytes);
                 tc::tma_load_2d(sbase + Lay::kQ + qs * Lay::kQBytes, &tmap_q, 0, t0 * HI, qfull_bar(qs));
                 ++q_issued;
-                for (int kt = 0; kt < ntile; ++kt) {
-                    if (!tc::mbar_wait(empty_bar(stage), phase ^ 1, kWaitLimitNs)) { ok = false; break; }
+                for (int st = 0; st < nstep; ++st) {
+                    if (!tc::mbar_wait_sleep(empty_bar(stage), phase ^ 1, kWaitLimitNs, kIssuerSleepNs)) {
+                        ok = false;
+                        break;
+                    }
                     tc::mbar_arrive_expect_tx(full_bar(stage), Lay::kTileBytes);
-                    tc::tma_load_2d(sbase + Lay::kKeys + stage * Lay::kTileBytes, &tmap_k, 0, kt * kTileM,
+                    tc::tma_load_2d(sbase + Lay::kKeys + stage * Lay::kTileBytes, &tmap_k, 0, st * kStepKeys,
                                     full_bar(stage));
                     ++n_issued;
                     if (++stage == kStages) { stage = 0; phase ^= 1; }
@@ -180,25 +205,36 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const __grid_co
                 const int qb = nb - 1 - i;
                 const int t0 = row_begin + qb * NQ;
                 const int t_hi = min(t0 + NQ, row_end) - 1;
-                const int ntile = t_hi / kTileM + 1;
+                const int nstep = t_hi / kStepKeys + 1;
                 const int qs = bi & 1;
-                if (!tc::mbar_wait(qfull_bar(qs), (bi >> 1) & 1, kWaitLimitNs)) { ok = false; break; }
+                if (!tc::mbar_wait_sleep(qfull_bar(qs), (bi >> 1) & 1, kWaitLimitNs, kIssuerSleepNs)) {
+                    ok = false;
+                    break;
+                }
                 tc::tc_fence_after();
                 const uint32_t qaddr = sbase + Lay::kQ + qs * Lay::kQBytes;
-                for (int kt = 0; kt < ntile; ++kt, ++it) {
-                    const int buf = it & 1;
-                    if (!tc::mbar_wait(tempty_bar(buf), ((it >> 1) & 1) ^ 1, kWaitLimitNs)) { ok = false; break; }
-                    if (!tc::mbar_wait(full_bar(stage), phase, kWaitLimitNs)) { ok = false; break; }
+                for (int st = 0; st < nstep; ++st, ++it) {
+                    const int pr = it % kPairs;
+                    if (!tc::mbar_wait_sleep(tempty_bar(pr), ((it / kPairs) & 1) ^ 1, kWaitLimitNs,
+                                             kIssuerSleepNs) ||
+                        !tc::mbar_wait_sleep(full_bar(stage), phase, kWaitLimitNs, kIssuerSleepNs)) {
+                        ok = false;
+                        break;
+                    }
                     tc::tc_fence_after();
                     const uint32_t kaddr = sbase + Lay::kKeys + stage * Lay::kTileBytes;
-                    const uint32_t d = tmem_base + (uint32_t)(buf * kTileN);
 #pragma unroll
-                    for (int ks = 0; ks < KSTEPS; ++ks) {
-                        tc::umma_f8(d, tc::smem_desc_kmajor(kaddr + ks * 32, DI),
-                                    tc::smem_desc_kmajor(qaddr + ks * 32, DI), IDESC, ks > 0 ? 1u : 0u);
+                    for (int h = 0; h < 2; ++h) {  // keys 0..127 and 128..255 of the step
+                        const uint32_t d = tmem_base + (uint32_t)((2 * pr + h) * kTileN);
+                        const uint32_t ka = kaddr + (uint32_t)(h * kTileM * DI);
+#pragma unroll
+                        for (int ks = 0; ks < KSTEPS; ++ks) {
+                            tc::umma_f8(d, tc::smem_desc_kmajor(ka + ks * 32, DI),
+                                        tc::smem_desc_kmajor(qaddr + ks * 32, DI), IDESC, ks > 0 ? 1u : 0u);
+                        }
                     }
                     tc::umma_commit(empty_bar(stage));
-                    tc::umma_commit(tfull_bar(buf));
+                    tc::umma_commit(tfull_bar(pr));
                     if (++stage == kStages) { stage = 0; phase ^= 1; }
                 }
                 tc::umma_commit(qempty_bar(qs));
@@ -211,72 +247,72 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_tc_kernel(const __grid_co
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        const int qw = warp & 3;        // TMEM lane quarter
-        const int cg = warp >> 2;       // 64-column group: queries cg*QPW ..
+        const int qw = warp & 3;          // TMEM lane quarter: keys 32*qw ..
+        const int cg = warp >> 2;         // column group: columns cg*CW ..
         const uint32_t lane_base = tmem_base + ((uint32_t)(qw * 32) << 16);
-        int it = 0, bi = 0;
+        int it = 0;
         bool ok = true;
-        for (int i = blockIdx.x; i < nb && ok; i += gridDim.x, ++bi) {
+        for (int i = blockIdx.x; i < nb && ok; i += gridDim.x) {
             const int qb = nb - 1 - i;
             const int t0 = row_begin + qb * NQ;
             const int t_hi = min(t0 + NQ, row_end) - 1;
-            const int ntile = t_hi / kTileM + 1;
-            const int wb = bi & 1;
-            {   // this block's head weights and query scales into shared memory
-                const int e = threadIdx.x;  // 0..511; (query, head) = e for e < 256
-                if (e < kTileN) {
-                    const int t = t0 + e / HI;
-                    w_s[wb * kTileN + e] = t <= t_hi ? __ldg(w + (size_t)t0 * HI + e) : 0.f;
-                }
-                if (e < NQ) sq_s[wb * 64 + e] = (t0 + e) <= t_hi ? __ldg(sq + t0 + e) : 0.f;
-                // All epilogue warps publish before any reads (bounded wait).  A
-                // warp can only rewrite this buffer two blocks later, after every
-                // warp has arrived for the block in between, i.e. finished this one.
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(wready_bar(wb));
-                if (!tc::mbar_wait(wready_bar(wb), (bi >> 1) & 1, kWaitLimitNs)) { ok = false; break; }
+            const int nstep = t_hi / kStepKeys + 1;
+            // this warp's query head weights, in registers for the whole block
+            float2 wv[CW / 2];
+#pragma unroll
+            for (int c = 0; c < CW; c += 2) {
+                const int t = t0 + (cg * CW + c) / HI;
+                wv[c / 2] = t <= t_hi ? __ldg(reinterpret_cast<const float2 *>(w + (size_t)t0 * HI + cg * CW + c))
+                                      : make_float2(0.f, 0.f);
             }
-            const float *wq = w_s + wb * kTileN + cg * 64;
-            for (int kt = 0; kt < ntile; ++kt, ++it) {
-                const int buf = it & 1;
-                const int s = kt * kTileM + qw * 32 + lane;
-                const float sks = s <= t_hi ? __ldg(sk + s) : 0.f;
-                if (!tc::mbar_wait(tfull_bar(buf), (it >> 1) & 1, kWaitLimitNs)) { ok = false; break; }
+            float sqv[QPW];
+#pragma unroll
+            for (int q = 0; q < QPW; ++q) {
+                const int t = t0 + (cg * CW) / HI + q;
+                sqv[q] = t <= t_hi ? __ldg(sq + t) : 0.f;
+            }
+            for (int st = 0; st < nstep; ++st, ++it) {
+                const int pr = it % kPairs;
+                if (!tc::mbar_wait(tfull_bar(pr), (it / kPairs) & 1, kWaitLimitNs)) { ok = false; break; }
                 tc::tc_fence_after();
-                float2 part[QPW][2];
 #pragma unroll
-                for (int q = 0; q < QPW; ++q) part[q][0] = part[q][1] = make_float2(0.f, 0.f);
+                for (int h = 0; h < 2; ++h) {
+                    const int buf = 2 * pr + h;
+                    const int s = st * kStepKeys + h * kTileM + qw * 32 + lane;
+                    const float sks = s <= t_hi ? __ldg(sk + s) : 0.f;
+                    float2 part[QPW][2];
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    float acc[32];
-                    tc::tmem_ld32(lane_base + (uint32_t)(buf * kTileN + cg * 64 + c * 32), acc);
-                    tc::tmem_wait_ld();
-                    if (c == 1) {  // accumulator read: hand it back to the MMA warp before the math
-                        tc::tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(tempty_bar(buf));
+                    for (int q = 0; q < QPW; ++q) part[q][0] = part[q][1] = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int c = 0; c < CW / 32; ++c) {
+                        float acc[32];
+                        tc::tmem_ld32(lane_base + (uint32_t)(buf * kTileN + cg * CW + c * 32), acc);
+                        tc::tmem_wait_ld();
+                        if (h == 1 && c == CW / 32 - 1) {  // the pair is read: hand it back before the math
+                            tc::tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) tc::mbar_arrive(tempty_bar(pr));
+                        }
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const int col = c * 32 + j;              // within this warp's CW columns
+                            const int q = col / HI;                  // compile-time after unrolling
+                            const int chain = (j >> 2) & 1;
+                            part[q][chain] = tc::ffma2(wv[col / 2],
+                                                       make_float2(fmaxf(acc[j], 0.f), fmaxf(acc[j + 1], 0.f)),
+                                                       part[q][chain]);
+                            part[q][chain] = tc::ffma2(wv[col / 2 + 1],
+                                                       make_float2(fmaxf(acc[j + 2], 0.f), fmaxf(acc[j + 3], 0.f)),
+                                                       part[q][chain]);
+                        }
                     }
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        const int col = c * 32 + j;              // within this warp's 64 columns
-                        const int q = col / HI;                  // compile-time after unrolling
-                        const int chain = (j >> 2) & 1;
-                        const float4 wv = *reinterpret_cast<const float4 *>(wq + col);
-                        part[q][chain] = tc::ffma2(make_float2(wv.x, wv.y),
-                                                   make_float2(fmaxf(acc[j], 0.f), fmaxf(acc[j + 1], 0.f)),
-                                                   part[q][chain]);
-                        part[q][chain] = tc::ffma2(make_float2(wv.z, wv.w),
-                                                   make_float2(fmaxf(acc[j + 2], 0.f), fmaxf(acc[j + 3], 0.f)),
-                                                   part[q][chain]);
-                    }
-                }
-#pragma unroll
-                for (int q = 0; q < QPW; ++q) {
-                    const int ql = cg * QPW + q;
-                    const int t = t0 + ql;
-                    if (t <= t_hi && s <= t) {
-                        const float v = (part[q][0].x + part[q][1].x) + (part[q][0].y + part[q][1].y);
-                        scores[(size_t)(t - row_begin) * ld + s] = v * sq_s[wb * 64 + ql] * sks;
+                    for (int q = 0; q < QPW; ++q) {
+                        const int t = t0 + (cg * CW) / HI + q;
+                        if (t <= t_hi && s <= t) {
+                            const float v = (part[q][0].x + part[q][1].x) + (part[q][0].y + part[q][1].y);
+                            scores[(size_t)(t - row_begin) * ld + s] = v * sqv[q] * sks;
+                        }
                     }
                 }
             }
@@ -332,7 +368,7 @@ template <int HI, int DI>
 cudaError_t launch_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8, const float *sk, int L,
                       int row_begin, int n_rows, float *scores, int64_t ld, cudaStream_t stream) {
     CUtensorMap mk, mq;
-    if (!make_map(&mk, k8, (uint64_t)L, DI, kTileM)) return cudaErrorInvalidValue;
+    if (!make_map(&mk, k8, (uint64_t)L, DI, kStepKeys)) return cudaErrorInvalidValue;
     if (!make_map(&mq, q8, (uint64_t)L * HI, DI, kTileN)) return cudaErrorInvalidValue;
     constexpr int NQ = kTileN / HI;
     const int nb = (n_rows + NQ - 1) / NQ;
@@ -341,7 +377,8 @@ cudaError_t launch_tc(const uint8_t *q8, const float *sq, const float *w, const 
     constexpr int smem = Layout<DI>::kAlloc > 116 * 1024 ? Layout<DI>::kAlloc : 116 * 1024;
     cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<HI, DI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    indexer_tc_kernel<HI, DI><<<grid, kThreads, smem, stream>>>(mk, mq, sq, w, sk, row_begin, n_rows, scores, ld);
+    indexer_tc_kernel<HI, DI><<<grid, EpiShape<HI>::kThreads, smem, stream>>>(mk, mq, sq, w, sk, row_begin, n_rows,
+                                                                             scores, ld);
     return cudaGetLastError();
 }
 

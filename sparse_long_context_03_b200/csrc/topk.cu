@@ -13,16 +13,17 @@
 //
 // One CTA owns one row; three passes over the row (the first from HBM, the
 // other two normally from L2):
-//   1. the row's key range [kmin, kmax];
+//   1. the row's value range [vmin, vmax];
 //   2. a histogram over 2048 linear buckets of that range (a monotone map,
 //      so bucket order is key order; scores spread over many buckets, which
 //      keeps shared-memory atomics free of hot spots);
 //   3. an ordered collect: entries in buckets above the threshold bucket Bt
 //      are winners, written in index order to a shared list A; entries in Bt
 //      are candidates, written in index order (key, index) to a list C.
-// T is then found inside C by a small radix select in shared memory, the
-// chosen candidates are compacted (still in index order), and A and the
-// chosen candidates are merged into the output by binary search.
+// The chosen candidates (by key, then index) are found by direct ranking when
+// there are few of them, by a small radix select in shared memory otherwise,
+// and compacted in index order; A and the chosen candidates are merged into
+// the output by binary search.  Only candidates are turned into keys.
 // If Bt holds more candidates than fit in shared memory (massive exact ties),
 // the row falls back to a radix select over the whole row (11/11/10-bit
 // passes) followed by an ordered compaction: slower, same result.
@@ -37,7 +38,8 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kNB = 2048;          // linear buckets (pass 2) and radix bins
 constexpr int kCap = 6144;         // candidates kept in shared memory
-constexpr int kVec = 4;            // consecutive entries per thread per chunk
+constexpr int kSmallCand = 256;    // up to this many candidates are ranked directly
+constexpr int kVec = 16;           // consecutive entries per thread per chunk (4 x float4 in flight)
 constexpr int kChunk = kThreads * kVec;
 
 struct TopkSmem {
@@ -57,31 +59,43 @@ __device__ __forceinline__ int row_length(const int32_t *row_len, int r, int row
     return n < 0 ? 0 : (n > max_len ? max_len : n);
 }
 
-// Load entries i0..i0+3 (fewer at the tail) as keys; absent entries get 0.
-__device__ __forceinline__ int load4(const float *row, int i0, int n, uint32_t (&key)[kVec]) {
+// Load entries i0..i0+kVec-1 (fewer at the tail); absent entries get 0.
+// A full group is four independent 16-byte loads issued back to back.
+__device__ __forceinline__ int load_vals(const float *row, int i0, int n, float (&x)[kVec]) {
     if (i0 + kVec <= n) {
-        const float4 v = __ldg(reinterpret_cast<const float4 *>(row + i0));
-        key[0] = order_key(v.x);
-        key[1] = order_key(v.y);
-        key[2] = order_key(v.z);
-        key[3] = order_key(v.w);
+        float4 v[kVec / 4];
+#pragma unroll
+        for (int q = 0; q < kVec / 4; ++q) v[q] = __ldg(reinterpret_cast<const float4 *>(row + i0) + q);
+#pragma unroll
+        for (int q = 0; q < kVec / 4; ++q) {
+            x[4 * q + 0] = v[q].x;
+            x[4 * q + 1] = v[q].y;
+            x[4 * q + 2] = v[q].z;
+            x[4 * q + 3] = v[q].w;
+        }
         return kVec;
     }
     int m = 0;
 #pragma unroll
     for (int j = 0; j < kVec; ++j) {
-        key[j] = (i0 + j < n) ? order_key(__ldg(row + i0 + j)) : 0u;
+        x[j] = (i0 + j < n) ? __ldg(row + i0 + j) : 0.f;
         m += (i0 + j < n);
     }
-    return m < 0 ? 0 : m;
+    return m;
 }
 
-__device__ __forceinline__ uint32_t bucket_of(uint32_t key, uint32_t kmin, float scale) {
-    const uint32_t b = __float2uint_rz(__fmul_rn(__uint2float_rn(key - kmin), scale));
+// Bucket of a score in [vmin, vmax]: rounded subtraction and multiplication
+// by a positive scale are monotone, and so is truncation, so bucket order is
+// score order (-0.0 and +0.0 share a bucket).  The explicit _rn intrinsics
+// keep the compiler from contracting the two steps differently in the two
+// passes that must agree.
+__device__ __forceinline__ uint32_t bucket_of(float x, float vmin, float scale) {
+    const uint32_t b = __float2uint_rz(__fmul_rn(__fsub_rn(x, vmin), scale));
     return b < (uint32_t)kNB ? b : (uint32_t)(kNB - 1);
 }
 
-// Exclusive block scan of one packed value per thread (two 16-bit counters).
+// Exclusive block scan of one packed value per thread (two 16-bit counters;
+// a chunk has kChunk = 8192 entries, so neither counter overflows).
 // Returns the exclusive prefix; *total gets the block total.  Two barriers.
 __device__ __forceinline__ uint32_t block_scan_packed(uint32_t v, uint32_t *red, uint32_t *total) {
     const int lane = lane_id(), warp = threadIdx.x >> 5;
@@ -227,47 +241,58 @@ __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__rest
         return;
     }
 
-    // ---- pass 1: key range
-    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    // ---- pass 1: value range
+    float vmin = INFINITY, vmax = -INFINITY;
     for (int i0 = tid * kVec; i0 < n; i0 += kChunk) {
-        uint32_t key[kVec];
-        const int m = load4(row, i0, n, key);
+        float x[kVec];
+        const int m = load_vals(row, i0, n, x);
 #pragma unroll
         for (int j = 0; j < kVec; ++j) {
             if (j < m) {
-                kmin = min(kmin, key[j]);
-                kmax = max(kmax, key[j]);
+                vmin = fminf(vmin, x[j]);
+                vmax = fmaxf(vmax, x[j]);
             }
         }
     }
-    kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
-    kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        vmin = fminf(vmin, __shfl_xor_sync(0xFFFFFFFFu, vmin, o));
+        vmax = fmaxf(vmax, __shfl_xor_sync(0xFFFFFFFFu, vmax, o));
+    }
+    float *fred = reinterpret_cast<float *>(sm.red);
     if (lane == 0) {
-        sm.red[warp] = kmin;
-        sm.red[kWarps + warp] = kmax;
+        fred[warp] = vmin;
+        fred[kWarps + warp] = vmax;
     }
     for (int i = tid; i < kNB; i += kThreads) sm.hist[i] = 0;
     __syncthreads();
-    kmin = sm.red[0];
-    kmax = sm.red[kWarps];
+    vmin = fred[0];
+    vmax = fred[kWarps];
 #pragma unroll
     for (int w = 1; w < kWarps; ++w) {
-        kmin = min(kmin, sm.red[w]);
-        kmax = max(kmax, sm.red[kWarps + w]);
+        vmin = fminf(vmin, fred[w]);
+        vmax = fmaxf(vmax, fred[kWarps + w]);
     }
-    if (kmin == kmax) {  // every entry ties: the k lowest indices
+    __syncthreads();
+    if (vmin == vmax) {  // every entry ties: the k lowest indices
         for (int i = tid; i < k; i += kThreads) out[i] = i;
         return;
     }
-    const float scale = (float)kNB / ((float)(kmax - kmin) + 1.0f);
+    const float range = vmax - vmin;
+    if (!(range < INFINITY)) {  // span overflows fp32: exact slow path
+        topk_row_radix(row, n, k, out, sm);
+        return;
+    }
+    // slightly below kNB / range so that vmax itself maps below kNB
+    const float scale = __fdiv_rn((float)kNB * 0.99999f, range);
 
     // ---- pass 2: bucket histogram
     for (int i0 = tid * kVec; i0 < n; i0 += kChunk) {
-        uint32_t key[kVec];
-        const int m = load4(row, i0, n, key);
+        float x[kVec];
+        const int m = load_vals(row, i0, n, x);
 #pragma unroll
         for (int j = 0; j < kVec; ++j)
-            if (j < m) atomicAdd(&sm.hist[bucket_of(key[j], kmin, scale)], 1u);
+            if (j < m) atomicAdd(&sm.hist[bucket_of(x[j], vmin, scale)], 1u);
     }
     __syncthreads();
     find_threshold_bin(sm.hist, (uint32_t)k, sm.red, sm.bcast);
@@ -286,13 +311,13 @@ __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__rest
     uint32_t run_a = 0, run_c = 0;
     for (int base = 0; base < n; base += kChunk) {
         const int i0 = base + tid * kVec;
-        uint32_t key[kVec] = {0u, 0u, 0u, 0u};
-        const int m = i0 < n ? load4(row, i0, n, key) : 0;
+        float x[kVec] = {};
+        const int m = i0 < n ? load_vals(row, i0, n, x) : 0;
         uint32_t cls[kVec];
         uint32_t na = 0, nc = 0;
 #pragma unroll
         for (int j = 0; j < kVec; ++j) {
-            const uint32_t b = bucket_of(key[j], kmin, scale);
+            const uint32_t b = bucket_of(x[j], vmin, scale);
             cls[j] = j >= m ? 0u : (b > Bt ? 2u : (b == Bt ? 1u : 0u));
             na += cls[j] == 2u;
             nc += cls[j] == 1u;
@@ -304,7 +329,7 @@ __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__rest
         for (int j = 0; j < kVec; ++j) {
             if (cls[j] == 2u) alist[pa++] = i0 + j;
             if (cls[j] == 1u) {
-                sm.ckey[pc] = key[j];
+                sm.ckey[pc] = order_key(x[j]);
                 sm.cidx[pc] = i0 + j;
                 ++pc;
             }
@@ -314,24 +339,44 @@ __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__rest
     }
     __syncthreads();
 
-    // ---- threshold key inside the candidates, then keep the chosen ones
-    uint32_t T, quota;
-    select_in_candidates(sm, (int)cnt, need, T, quota);
-    uint32_t run_g = 0, run_e = 0;
-    for (int base = 0; base < (int)cnt; base += kThreads) {
-        const int i = base + tid;
-        const uint32_t key = i < (int)cnt ? sm.ckey[i] : 0u;
-        const int32_t ix = i < (int)cnt ? sm.cidx[i] : 0;
-        const bool gt = i < (int)cnt && key > T;
-        const bool eq = i < (int)cnt && key == T;
+    // ---- choose `need` candidates: larger key first, lower index on ties
+    if (cnt <= (uint32_t)kSmallCand) {
+        // Direct ranking: candidate i is chosen iff fewer than `need`
+        // candidates beat it (larger key, or equal key and lower index).
+        // Candidates sit in index order, so "lower index" is "earlier slot".
+        const int i = tid;
+        const bool act = i < (int)cnt;
+        const uint32_t ki = act ? sm.ckey[i] : 0u;
+        const int32_t ix = act ? sm.cidx[i] : 0;
+        uint32_t rank = 0;
+        for (int j = 0; j < (int)cnt; ++j) {
+            const uint32_t kj = sm.ckey[j];
+            rank += (kj > ki) || (kj == ki && j < i);
+        }
+        const bool chosen = act && rank < need;
         uint32_t tot;
-        const uint32_t ex = block_scan_packed((gt ? 1u : 0u) | (eq ? 0x10000u : 0u), sm.red, &tot);
-        const uint32_t gb = run_g + (ex & 0xFFFFu), eb = run_e + (ex >> 16);
-        // positions only move left and this chunk was read before the scan's barriers
-        if (gt || (eq && eb < quota)) sm.cidx[gb + min(eb, quota)] = ix;
-        run_g += tot & 0xFFFFu;
-        run_e += tot >> 16;
+        const uint32_t ex = block_scan_packed(chosen ? 1u : 0u, sm.red, &tot);
+        if (chosen) sm.cidx[ex] = ix;  // ex <= i, and slot i was read above
         __syncthreads();
+    } else {
+        uint32_t T, quota;
+        select_in_candidates(sm, (int)cnt, need, T, quota);
+        uint32_t run_g = 0, run_e = 0;
+        for (int base = 0; base < (int)cnt; base += kThreads) {
+            const int i = base + tid;
+            const uint32_t key = i < (int)cnt ? sm.ckey[i] : 0u;
+            const int32_t ix = i < (int)cnt ? sm.cidx[i] : 0;
+            const bool gt = i < (int)cnt && key > T;
+            const bool eq = i < (int)cnt && key == T;
+            uint32_t tot;
+            const uint32_t ex = block_scan_packed((gt ? 1u : 0u) | (eq ? 0x10000u : 0u), sm.red, &tot);
+            const uint32_t gb = run_g + (ex & 0xFFFFu), eb = run_e + (ex >> 16);
+            // positions only move left and this chunk was read before the scan's barriers
+            if (gt || (eq && eb < quota)) sm.cidx[gb + min(eb, quota)] = ix;
+            run_g += tot & 0xFFFFu;
+            run_e += tot >> 16;
+            __syncthreads();
+        }
     }
 
     // ---- merge the two ascending lists into the output
