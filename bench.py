@@ -169,11 +169,11 @@ class PrefillBench:
             if ev is not None:
                 a = torch.cuda.Event(enable_timing=True)
                 a.record(self.stream)
-            dsa.indexer_scores(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], r0, n, p.scores[:n])
+            dsa.indexer_scores(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], r0, n, p.scores[:n], row_stats=p.row_stats)
             if ev is not None:
                 b = torch.cuda.Event(enable_timing=True)
                 b.record(self.stream)
-            dsa.topk(p.scores[:n], r0, n, c.k, p.idx[r0:r0 + n], max_len=r0 + n, ws=p.ws)
+            dsa.topk(p.scores[:n], r0, n, c.k, p.idx[r0:r0 + n], max_len=r0 + n, ws=p.ws, row_stats=p.row_stats)
             if ev is not None:
                 e = torch.cuda.Event(enable_timing=True)
                 e.record(self.stream)

@@ -91,13 +91,19 @@ DSA_API dsa_status_t dsa_check_device_error(void);
  *            ld_scores >= row_begin + n_rows and ld_scores % 4 == 0.
  *   q8, k8 must be 16-byte aligned (they are read by the tensor-memory
  *   accelerator).
+ *   row_stats  optional (NULL to skip): device buffer of
+ *            dsa_row_stats_bytes(n_rows) bytes that receives, per row, the
+ *            range of the scores just written.  Its layout is private to the
+ *            library; passing it to dsa_topk for the same rows lets the top-k
+ *            skip its own pass over the row to find that range.
  * Supported: dI in {32, 64, 128}; HI in {4, 8, 16, 32, 64}.
  * All scale factors must be positive (they commute with the ReLU).
  * ------------------------------------------------------------------------ */
+DSA_API size_t dsa_row_stats_bytes(int n_rows);
 DSA_API dsa_status_t dsa_indexer_scores(const uint8_t *q8, const float *q_scale, const float *w,
                                 const uint8_t *k8, const float *k_scale,
                                 int L, int HI, int dI, int row_begin, int n_rows,
-                                float *scores, int64_t ld_scores, void *stream);
+                                float *scores, int64_t ld_scores, void *row_stats, void *stream);
 
 /* ------------------------------------------------------------------------
  * Per-row top-k selection.
@@ -114,13 +120,15 @@ DSA_API dsa_status_t dsa_indexer_scores(const uint8_t *q8, const float *q_scale,
  *   max_len  upper bound of every n_r (the host sizes grids with it);
  *            ld_scores >= max_len and ld_scores % 4 == 0; scores 16-byte aligned.
  * Supported: 1 <= k <= 40000 (a row's winners are staged in shared memory).
+ *   row_stats  NULL, or the buffer dsa_indexer_scores filled for exactly
+ *            these rows (same row_begin / n_rows, scores unchanged since).
  *   ws       device workspace of at least dsa_topk_workspace_size() bytes
  *            (may be NULL when that size is 0).
  * ------------------------------------------------------------------------ */
 DSA_API size_t dsa_topk_workspace_size(int n_rows, int max_len, int k);
 DSA_API dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, int row_begin, int n_rows,
                       const int32_t *row_len, int max_len, int k, int32_t *idx,
-                      void *ws, size_t ws_bytes, void *stream);
+                      const void *row_stats, void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
  * Sparse GQA attention (prefill), one chunk of query rows.

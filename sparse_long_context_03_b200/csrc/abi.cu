@@ -67,20 +67,26 @@ dsa_status_t dsa_check_device_error(void) {
     return flag ? DSA_ERR_TIMEOUT : DSA_OK;
 }
 
+size_t dsa_row_stats_bytes(int n_rows) { return n_rows > 0 ? (size_t)n_rows * 8 * sizeof(float) : 0; }
+
 dsa_status_t dsa_indexer_scores(const uint8_t *q8, const float *q_scale, const float *w, const uint8_t *k8,
                                 const float *k_scale, int L, int HI, int dI, int row_begin, int n_rows,
-                                float *scores, int64_t ld_scores, void *stream) {
+                                float *scores, int64_t ld_scores, void *row_stats, void *stream) {
     if (L < 1 || row_begin < 0 || n_rows < 0 || (int64_t)row_begin + n_rows > L) return DSA_ERR_INVALID_ARG;
     if (!dsa::indexer_shape_supported(HI, dI)) return DSA_ERR_UNSUPPORTED_SHAPE;
     if (n_rows == 0) return DSA_OK;
     if (!q8 || !q_scale || !w || !k8 || !k_scale || !scores) return DSA_ERR_INVALID_ARG;
     if (ld_scores < (int64_t)row_begin + n_rows || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(q8) | reinterpret_cast<uintptr_t>(k8)) % 16 != 0) return DSA_ERR_INVALID_ARG;
+    float *stats = static_cast<float *>(row_stats);
     if (dsa::indexer_tc_supported(HI, dI))
         return cuda_status(dsa::launch_indexer_prefill_tc(q8, q_scale, w, k8, k_scale, L, HI, dI, row_begin, n_rows,
-                                                          scores, ld_scores, as_stream(stream)));
-    return cuda_status(dsa::launch_indexer_prefill_mma(q8, q_scale, w, k8, k_scale, HI, dI, row_begin, n_rows,
-                                                       scores, ld_scores, as_stream(stream)));
+                                                          scores, ld_scores, stats, as_stream(stream)));
+    cudaError_t e = dsa::launch_indexer_prefill_mma(q8, q_scale, w, k8, k_scale, HI, dI, row_begin, n_rows, scores,
+                                                    ld_scores, as_stream(stream));
+    if (e == cudaSuccess && stats != nullptr)
+        e = dsa::launch_row_stats(scores, ld_scores, row_begin, n_rows, stats, as_stream(stream));
+    return cuda_status(e);
 }
 
 size_t dsa_topk_workspace_size(int n_rows, int max_len, int k) {
@@ -89,7 +95,8 @@ size_t dsa_topk_workspace_size(int n_rows, int max_len, int k) {
 }
 
 dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, int row_begin, int n_rows, const int32_t *row_len,
-                      int max_len, int k, int32_t *idx, void *ws, size_t ws_bytes, void *stream) {
+                      int max_len, int k, int32_t *idx, const void *row_stats, void *ws, size_t ws_bytes,
+                      void *stream) {
     if (n_rows < 0 || row_begin < 0 || k < 1 || max_len < 0) return DSA_ERR_INVALID_ARG;
     if (row_len == nullptr && (int64_t)row_begin + n_rows > max_len) return DSA_ERR_INVALID_ARG;
     if (n_rows == 0) return DSA_OK;
@@ -99,8 +106,8 @@ dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, int row_begin, int
     if (!dsa::topk_k_supported(k)) return DSA_ERR_UNSUPPORTED_SHAPE;
     const size_t need = dsa::topk_workspace_bytes(n_rows, max_len, k);
     if (ws_bytes < need || (need > 0 && ws == nullptr)) return DSA_ERR_WORKSPACE;
-    return cuda_status(dsa::launch_topk(scores, ld_scores, row_begin, n_rows, row_len, max_len, k, idx, ws,
-                                        ws_bytes, as_stream(stream)));
+    return cuda_status(dsa::launch_topk(scores, ld_scores, row_begin, n_rows, row_len, max_len, k, idx,
+                                        static_cast<const float *>(row_stats), ws, ws_bytes, as_stream(stream)));
 }
 
 dsa_status_t dsa_sparse_gqa_prefill(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const int32_t *idx,
@@ -210,7 +217,7 @@ dsa_status_t dsa_sparse_gqa_decode(const uint16_t *q, const uint8_t *q8, const f
     cudaError_t e = dsa::launch_indexer_decode(q8, q_scale, w, k8_cache, k_scale_cache, block_table, max_pages,
                                                num_pages, seq_lens, max_seq_len, B, HI, dI, scores, L.ld, s);
     if (e != cudaSuccess) return cuda_status(e);
-    e = dsa::launch_topk(scores, L.ld, 0, B, seq_lens, max_seq_len, k, idx, base + L.topk_off,
+    e = dsa::launch_topk(scores, L.ld, 0, B, seq_lens, max_seq_len, k, idx, nullptr, base + L.topk_off,
                          dsa::topk_workspace_bytes(B, max_seq_len, k), s);
     if (e != cudaSuccess) return cuda_status(e);
     e = dsa::launch_sparse_decode(q, k_cache, v_cache, block_table, max_pages, num_pages, seq_lens, idx, B, Hq, Hkv,

@@ -226,7 +226,37 @@ bool dispatch_shape(int HI, int dI, F &&launch) {
     }
 }
 
+// Row value range of already written prefill score rows (one warp per row),
+// in the row-statistics layout the top-k reads: four (min, max) partials per
+// row; here the first carries the whole row and the others are empty.
+__global__ void __launch_bounds__(256) row_stats_kernel(const float *__restrict__ scores, int64_t ld, int row_begin,
+                                                        int n_rows, float *__restrict__ row_stats) {
+    const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= n_rows) return;
+    const int lane = lane_id(), n = row_begin + r + 1;
+    const float *row = scores + (size_t)r * ld;
+    float lo = INFINITY, hi = -INFINITY;
+    for (int i = lane; i < n; i += 32) {
+        const float v = __ldg(row + i);
+        lo = fminf(lo, v);
+        hi = fmaxf(hi, v);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+    }
+    if (lane < 8) row_stats[(size_t)r * 8 + lane] = lane == 0 ? lo : (lane == 1 ? hi : ((lane & 1) ? -INFINITY : INFINITY));
+}
+
 }  // namespace
+
+cudaError_t launch_row_stats(const float *scores, int64_t ld, int row_begin, int n_rows, float *row_stats,
+                             cudaStream_t stream) {
+    if (n_rows == 0) return cudaSuccess;
+    row_stats_kernel<<<(n_rows + 7) / 8, 256, 0, stream>>>(scores, ld, row_begin, n_rows, row_stats);
+    return cudaGetLastError();
+}
 
 bool indexer_shape_supported(int HI, int dI) {
     return (HI == 4 || HI == 8 || HI == 16 || HI == 32 || HI == 64) && (dI == 32 || dI == 64 || dI == 128);

@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(EpiShape<HI>::kThreads, 1) indexer_tc_kernel(c
                                                                  const float *__restrict__ w,
                                                                  const float *__restrict__ sk, int row_begin,
                                                                  int n_rows, float *__restrict__ scores,
-                                                                 int64_t ld) {
+                                                                 int64_t ld, float *__restrict__ row_stats) {
     using Lay = Layout<DI>;
     using ES = EpiShape<HI>;
     constexpr int kEpiWarps = ES::kEpiWarps, kProducerWarp = ES::kProducerWarp, kMmaWarp = ES::kMmaWarp;
@@ -265,11 +265,13 @@ __global__ void __launch_bounds__(EpiShape<HI>::kThreads, 1) indexer_tc_kernel(c
                 wv[c / 2] = t <= t_hi ? __ldg(reinterpret_cast<const float2 *>(w + (size_t)t0 * HI + cg * CW + c))
                                       : make_float2(0.f, 0.f);
             }
-            float sqv[QPW];
+            float sqv[QPW], vlo[QPW], vhi[QPW];
 #pragma unroll
             for (int q = 0; q < QPW; ++q) {
                 const int t = t0 + (cg * CW) / HI + q;
                 sqv[q] = t <= t_hi ? __ldg(sq + t) : 0.f;
+                vlo[q] = INFINITY;
+                vhi[q] = -INFINITY;
             }
             for (int st = 0; st < nstep; ++st, ++it) {
                 const int pr = it % kPairs;
@@ -311,8 +313,28 @@ __global__ void __launch_bounds__(EpiShape<HI>::kThreads, 1) indexer_tc_kernel(c
                         const int t = t0 + (cg * CW) / HI + q;
                         if (t <= t_hi && s <= t) {
                             const float v = (part[q][0].x + part[q][1].x) + (part[q][0].y + part[q][1].y);
-                            scores[(size_t)(t - row_begin) * ld + s] = v * sqv[q] * sks;
+                            const float score = v * sqv[q] * sks;
+                            scores[(size_t)(t - row_begin) * ld + s] = score;
+                            vlo[q] = fminf(vlo[q], score);
+                            vhi[q] = fmaxf(vhi[q], score);
                         }
+                    }
+                }
+            }
+            if (row_stats != nullptr && ok) {
+                // per-(row, lane quarter) range of the scores just written
+#pragma unroll
+                for (int q = 0; q < QPW; ++q) {
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        vlo[q] = fminf(vlo[q], __shfl_xor_sync(0xFFFFFFFFu, vlo[q], o));
+                        vhi[q] = fmaxf(vhi[q], __shfl_xor_sync(0xFFFFFFFFu, vhi[q], o));
+                    }
+                    const int t = t0 + (cg * CW) / HI + q;
+                    if (lane == 0 && t <= t_hi) {
+                        float *st8 = row_stats + (size_t)(t - row_begin) * 8;
+                        st8[2 * qw] = vlo[q];
+                        st8[2 * qw + 1] = vhi[q];
                     }
                 }
             }
@@ -366,7 +388,7 @@ int sm_count() {
 
 template <int HI, int DI>
 cudaError_t launch_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8, const float *sk, int L,
-                      int row_begin, int n_rows, float *scores, int64_t ld, cudaStream_t stream) {
+                      int row_begin, int n_rows, float *scores, int64_t ld, float *row_stats, cudaStream_t stream) {
     CUtensorMap mk, mq;
     if (!make_map(&mk, k8, (uint64_t)L, DI, kStepKeys)) return cudaErrorInvalidValue;
     if (!make_map(&mq, q8, (uint64_t)L * HI, DI, kTileN)) return cudaErrorInvalidValue;
@@ -378,7 +400,7 @@ cudaError_t launch_tc(const uint8_t *q8, const float *sq, const float *w, const 
     cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<HI, DI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     indexer_tc_kernel<HI, DI><<<grid, EpiShape<HI>::kThreads, smem, stream>>>(mk, mq, sq, w, sk, row_begin, n_rows,
-                                                                             scores, ld);
+                                                                             scores, ld, row_stats);
     return cudaGetLastError();
 }
 
@@ -390,14 +412,14 @@ bool indexer_tc_supported(int HI, int dI) {
 
 cudaError_t launch_indexer_prefill_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
                                       const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
-                                      float *scores, int64_t ld, cudaStream_t stream) {
+                                      float *scores, int64_t ld, float *row_stats, cudaStream_t stream) {
     if (n_rows == 0) return cudaSuccess;
     auto by_di = [&](auto hi) -> cudaError_t {
         constexpr int H = decltype(hi)::value;
         switch (dI) {
-            case 32: return launch_tc<H, 32>(q8, sq, w, k8, sk, L, row_begin, n_rows, scores, ld, stream);
-            case 64: return launch_tc<H, 64>(q8, sq, w, k8, sk, L, row_begin, n_rows, scores, ld, stream);
-            case 128: return launch_tc<H, 128>(q8, sq, w, k8, sk, L, row_begin, n_rows, scores, ld, stream);
+            case 32: return launch_tc<H, 32>(q8, sq, w, k8, sk, L, row_begin, n_rows, scores, ld, row_stats, stream);
+            case 64: return launch_tc<H, 64>(q8, sq, w, k8, sk, L, row_begin, n_rows, scores, ld, row_stats, stream);
+            case 128: return launch_tc<H, 128>(q8, sq, w, k8, sk, L, row_begin, n_rows, scores, ld, row_stats, stream);
             default: return cudaErrorInvalidValue;
         }
     };

@@ -12,6 +12,8 @@ bool indexer_shape_supported(int HI, int dI);
 cudaError_t launch_indexer_prefill_mma(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
                                        const float *sk, int HI, int dI, int row_begin, int n_rows, float *scores,
                                        int64_t ld, cudaStream_t stream);
+cudaError_t launch_row_stats(const float *scores, int64_t ld, int row_begin, int n_rows, float *row_stats,
+                             cudaStream_t stream);
 cudaError_t launch_indexer_decode(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8c,
                                   const float *skc, const int32_t *block_table, int max_pages, int num_pages,
                                   const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI, float *scores,
@@ -21,14 +23,15 @@ cudaError_t launch_indexer_decode(const uint8_t *q8, const float *sq, const floa
 bool indexer_tc_supported(int HI, int dI);
 cudaError_t launch_indexer_prefill_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
                                       const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
-                                      float *scores, int64_t ld, cudaStream_t stream);
+                                      float *scores, int64_t ld, float *row_stats, cudaStream_t stream);
 cudaError_t indexer_tc_take_error(unsigned int *flag);
 
 // topk.cu
 size_t topk_workspace_bytes(int n_rows, int max_len, int k);
 bool topk_k_supported(int k);
 cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_rows, const int32_t *row_len,
-                        int max_len, int k, int32_t *idx, void *ws, size_t ws_bytes, cudaStream_t stream);
+                        int max_len, int k, int32_t *idx, const float *row_stats, void *ws, size_t ws_bytes,
+                        cudaStream_t stream);
 
 // attention.cu
 bool attention_shape_supported(int Hq, int Hkv, int D);

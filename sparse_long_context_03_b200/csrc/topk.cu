@@ -13,7 +13,8 @@
 //
 // One CTA owns one row; three passes over the row (the first from HBM, the
 // other two normally from L2):
-//   1. the row's value range [vmin, vmax];
+//   1. the row's value range [vmin, vmax] -- skipped when the indexer already
+//      produced it (row statistics), so the histogram pass reads from HBM;
 //   2. a histogram over 2048 linear buckets of that range (a monotone map,
 //      so bucket order is key order; scores spread over many buckets, which
 //      keeps shared-memory atomics free of hot spots);
@@ -225,7 +226,8 @@ __device__ void topk_row_radix(const float *row, int n, int k, int32_t *out, Top
 
 __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__restrict__ scores, int64_t ld,
                                                             int row_begin, const int32_t *__restrict__ row_len,
-                                                            int max_len, int k, int32_t *__restrict__ idx) {
+                                                            int max_len, int k, int32_t *__restrict__ idx,
+                                                            const float *__restrict__ row_stats) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
     int32_t *alist = reinterpret_cast<int32_t *>(smem_raw + sizeof(TopkSmem));
@@ -241,8 +243,14 @@ __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__rest
         return;
     }
 
-    // ---- pass 1: value range
+    // ---- pass 1: value range (from the indexer's row statistics when given)
     float vmin = INFINITY, vmax = -INFINITY;
+    if (row_stats != nullptr) {
+        if (tid < 4) {
+            vmin = __ldg(row_stats + (size_t)r * 8 + 2 * tid);
+            vmax = __ldg(row_stats + (size_t)r * 8 + 2 * tid + 1);
+        }
+    } else
     for (int i0 = tid * kVec; i0 < n; i0 += kChunk) {
         float x[kVec];
         const int m = load_vals(row, i0, n, x);
@@ -407,13 +415,15 @@ __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__rest
 size_t topk_workspace_bytes(int, int, int) { return 0; }
 
 cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_rows, const int32_t *row_len,
-                        int max_len, int k, int32_t *idx, void *, size_t, cudaStream_t stream) {
+                        int max_len, int k, int32_t *idx, const float *row_stats, void *, size_t,
+                        cudaStream_t stream) {
     if (n_rows == 0) return cudaSuccess;
     const size_t smem = smem_bytes(k);
     if (smem > 220 * 1024) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    topk_rows_kernel<<<n_rows, kThreads, smem, stream>>>(scores, ld, row_begin, row_len, max_len, k, idx);
+    topk_rows_kernel<<<n_rows, kThreads, smem, stream>>>(scores, ld, row_begin, row_len, max_len, k, idx,
+                                                         row_stats);
     return cudaGetLastError();
 }
 

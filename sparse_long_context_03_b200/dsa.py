@@ -33,9 +33,10 @@ _SIGNATURES = {
     "dsa_version": ([], _I),
     "dsa_last_error_string": ([], ctypes.c_char_p),
     "dsa_check_device_error": ([], _I),
-    "dsa_indexer_scores": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P], _I),
+    "dsa_row_stats_bytes": ([_I], _SZ),
+    "dsa_indexer_scores": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P, _P], _I),
     "dsa_topk_workspace_size": ([_I, _I, _I], _SZ),
-    "dsa_topk": ([_P, _I64, _I, _I, _P, _I, _I, _P, _P, _SZ, _P], _I),
+    "dsa_topk": ([_P, _I64, _I, _I, _P, _I, _I, _P, _P, _P, _SZ, _P], _I),
     "dsa_sparse_gqa_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P], _I),
     "dsa_decode_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
     "dsa_sparse_gqa_decode": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _I,
@@ -119,15 +120,21 @@ def _need(t, dtype, ndim, name):
 # prefill
 # ---------------------------------------------------------------------------
 
-def indexer_scores(q8, q_scale, w, k8, k_scale, row_begin, n_rows, scores, stream=None):
+def row_stats_bytes(n_rows) -> int:
+    return int(lib().dsa_row_stats_bytes(int(n_rows)))
+
+
+def indexer_scores(q8, q_scale, w, k8, k_scale, row_begin, n_rows, scores, row_stats=None, stream=None):
     """dsa_indexer_scores: rows [row_begin, row_begin+n_rows) of the causal
-    lightning-indexer score matrix into ``scores`` [n_rows, ld] float32."""
+    lightning-indexer score matrix into ``scores`` [n_rows, ld] float32;
+    optionally the rows' value ranges into ``row_stats`` for dsa_topk."""
     _need(q8, torch.uint8, 3, "q8")
     _need(k8, torch.uint8, 2, "k8")
     _need(scores, torch.float32, 2, "scores")
     L, HI, dI = q8.shape
     _check(lib().dsa_indexer_scores(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), L, HI, dI,
-                                    int(row_begin), int(n_rows), _ptr(scores), scores.stride(0), _stream(stream)),
+                                    int(row_begin), int(n_rows), _ptr(scores), scores.stride(0), _ptr(row_stats),
+                                    _stream(stream)),
            "dsa_indexer_scores")
 
 
@@ -135,7 +142,7 @@ def topk_workspace_size(n_rows, max_len, k) -> int:
     return int(lib().dsa_topk_workspace_size(int(n_rows), int(max_len), int(k)))
 
 
-def topk(scores, row_begin, n_rows, k, idx, row_len=None, max_len=None, ws=None, stream=None):
+def topk(scores, row_begin, n_rows, k, idx, row_len=None, max_len=None, ws=None, row_stats=None, stream=None):
     """dsa_topk: per-row top-k (ascending indices, -1 padded) into idx [n_rows, k]."""
     _need(scores, torch.float32, 2, "scores")
     _need(idx, torch.int32, 2, "idx")
@@ -148,7 +155,7 @@ def topk(scores, row_begin, n_rows, k, idx, row_len=None, max_len=None, ws=None,
             raise DSAError(f"dsa_topk needs a {need}-byte workspace")
         ws_bytes = ws.numel() * ws.element_size()
     _check(lib().dsa_topk(_ptr(scores), scores.stride(0), int(row_begin), int(n_rows), _ptr(row_len), int(max_len),
-                          int(k), _ptr(idx), _ptr(ws), ws_bytes, _stream(stream)), "dsa_topk")
+                          int(k), _ptr(idx), _ptr(row_stats), _ptr(ws), ws_bytes, _stream(stream)), "dsa_topk")
 
 
 def sparse_gqa_prefill(Q, K, V, idx, row_begin, n_rows, k, sm_scale, O, lse=None, stream=None):
@@ -179,6 +186,7 @@ class PrefillPlan:
         self.idx = torch.empty(L, k, dtype=torch.int32, device=device)
         need = topk_workspace_size(self.chunk_rows, L, k)
         self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=device) if need else None
+        self.row_stats = torch.empty(row_stats_bytes(self.chunk_rows), dtype=torch.uint8, device=device)
 
     def chunks(self):
         for r0 in range(0, self.L, self.chunk_rows):
@@ -192,8 +200,9 @@ def prefill_forward(plan: PrefillPlan, q8, sq, w, k8, sk, Q, K, V, O, sm_scale=N
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(plan.D)
     for r0, n in plan.chunks():
-        indexer_scores(q8, sq, w, k8, sk, r0, n, plan.scores[:n], stream=stream)
-        topk(plan.scores[:n], r0, n, plan.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws, stream=stream)
+        indexer_scores(q8, sq, w, k8, sk, r0, n, plan.scores[:n], row_stats=plan.row_stats, stream=stream)
+        topk(plan.scores[:n], r0, n, plan.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws,
+             row_stats=plan.row_stats, stream=stream)
     sparse_gqa_prefill(Q, K, V, plan.idx, 0, plan.L, plan.k, sm_scale, O, lse, stream=stream)
 
 

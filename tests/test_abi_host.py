@@ -56,7 +56,7 @@ def test_indexer_rejects_bad_arguments(lib):
     def call(**kw):
         a = {**good, **kw}
         ptrs = [kw.get("p", BOGUS)] * 5
-        return f(*ptrs, a["L"], a["HI"], a["dI"], a["rb"], a["n"], kw.get("out", BOGUS), a["ld"], None)
+        return f(*ptrs, a["L"], a["HI"], a["dI"], a["rb"], a["n"], kw.get("out", BOGUS), a["ld"], None, None)
 
     assert call(HI=3) == UNSUPPORTED
     assert call(dI=48) == UNSUPPORTED
@@ -71,11 +71,11 @@ def test_indexer_rejects_bad_arguments(lib):
 
 def test_topk_rejects_bad_arguments(lib):
     f = lib.dsa_topk
-    assert f(BOGUS, 512, 0, 512, None, 512, 0, BOGUS, None, 0, None) == INVALID   # k < 1
-    assert f(BOGUS, 512, 100, 500, None, 512, 64, BOGUS, None, 0, None) == INVALID  # rows past max_len
-    assert f(BOGUS, 510, 0, 4, BOGUS, 512, 64, BOGUS, None, 0, None) == INVALID   # ld < max_len
-    assert f(None, 512, 0, 4, BOGUS, 512, 64, BOGUS, None, 0, None) == INVALID
-    assert f(BOGUS, 512, 0, 0, None, 512, 64, BOGUS, None, 0, None) == OK
+    assert f(BOGUS, 512, 0, 512, None, 512, 0, BOGUS, None, None, 0, None) == INVALID   # k < 1
+    assert f(BOGUS, 512, 100, 500, None, 512, 64, BOGUS, None, None, 0, None) == INVALID  # rows past max_len
+    assert f(BOGUS, 510, 0, 4, BOGUS, 512, 64, BOGUS, None, None, 0, None) == INVALID   # ld < max_len
+    assert f(None, 512, 0, 4, BOGUS, 512, 64, BOGUS, None, None, 0, None) == INVALID
+    assert f(BOGUS, 512, 0, 0, None, 512, 64, BOGUS, None, None, 0, None) == OK
 
 
 def test_attention_rejects_bad_arguments(lib):
@@ -109,3 +109,4 @@ def test_workspace_queries(lib):
     assert a > b > 32 * 131072 * 4
     assert lib.dsa_decode_attention_workspace_size(32, 32, 4, 128, 2048) > 0
     assert lib.dsa_topk_workspace_size(8, 1000, 0) == 0
+    assert lib.dsa_row_stats_bytes(100) == 100 * 32

@@ -163,7 +163,7 @@ def test_topk_signed_zeros_and_all_equal():
 # whole prefill chain, small
 # ----------------------------------------------------------------------------
 
-def run_prefill(cfg, d, chunk_rows=None, want_rows=(), lse=True):
+def run_prefill(cfg, d, chunk_rows=None, want_rows=(), lse=True, use_stats=True):
     """Run the chunked prefill exactly as the benchmark does; also copy out
     the score rows listed in want_rows as each chunk is produced."""
     L = d["q8"].shape[0]
@@ -173,20 +173,23 @@ def run_prefill(cfg, d, chunk_rows=None, want_rows=(), lse=True):
     want = sorted(want_rows)
     rows = {}
     for r0, n in plan.chunks():
-        dsa.indexer_scores(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], r0, n, plan.scores[:n])
+        dsa.indexer_scores(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], r0, n, plan.scores[:n],
+                           row_stats=plan.row_stats if use_stats else None)
         for t in want:
             if r0 <= t < r0 + n:
                 rows[t] = plan.scores[t - r0, : t + 1].cpu().numpy()
-        dsa.topk(plan.scores[:n], r0, n, cfg.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws)
+        dsa.topk(plan.scores[:n], r0, n, cfg.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws,
+                 row_stats=plan.row_stats if use_stats else None)
     dsa.sparse_gqa_prefill(d["Q"], d["K"], d["V"], plan.idx, 0, L, cfg.k, cfg.sm_scale, O, lse_t)
     torch.cuda.synchronize()
     return plan, O, lse_t, rows
 
 
-def test_prefill_chain_tiny_full():
+@pytest.mark.parametrize("use_stats", [True, False])
+def test_prefill_chain_tiny_full(use_stats):
     cfg = inputs.config(0)
     d = inputs.prefill_inputs(cfg)
-    plan, O, lse, _ = run_prefill(cfg, _gpu(d), chunk_rows=200)
+    plan, O, lse, _ = run_prefill(cfg, _gpu(d), chunk_rows=200, use_stats=use_stats)
     h = {k: H(v) for k, v in d.items()}
     I = oracle.indexer(h["q8"], h["sq"], h["w"], h["k8"], h["sk"])
     ref_idx = oracle.causal_topk(I, 0, cfg.k)
@@ -213,11 +216,12 @@ def test_prefill_chain_exact_inputs_bit_exact_indices():
     g = torch.Generator().manual_seed(1)
     for name, Hh in (("Q", cfg.Hq), ("K", cfg.Hkv), ("V", cfg.Hkv)):
         d[name] = (torch.randn(L, Hh, cfg.D, generator=g) * 0.5).to(torch.bfloat16)
-    plan, O, lse, _ = run_prefill(cfg, _gpu(d), chunk_rows=256)
     h = {k: H(v) for k, v in d.items()}
     I = oracle.indexer(h["q8"], h["sq"], h["w"], h["k8"], h["sk"])
     ref_idx = oracle.causal_topk(I, 0, cfg.k)
-    assert np.array_equal(plan.idx.cpu().numpy(), ref_idx)
+    for use_stats in (True, False):
+        plan, O, lse, _ = run_prefill(cfg, _gpu(d), chunk_rows=256, use_stats=use_stats)
+        assert np.array_equal(plan.idx.cpu().numpy(), ref_idx)
     Oref, lref = oracle.sparse_attention(h["Q"], h["K"], h["V"], ref_idx, 0, cfg.sm_scale)
     check_attention(O.float().cpu().numpy(), Oref, lse.cpu().numpy(), lref, "exact chain")
 
