@@ -28,6 +28,8 @@
 // If Bt holds more candidates than fit in shared memory (massive exact ties),
 // the row falls back to a radix select over the whole row (11/11/10-bit
 // passes) followed by an ordered compaction: slower, same result.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -224,6 +226,76 @@ __device__ void topk_row_radix(const float *row, int n, int k, int32_t *out, Top
     }
 }
 
+// Final step of one row: the shared lists hold, in index order, the n_above
+// winners (alist) and the cnt threshold-bucket candidates (ckey / cidx);
+// choose `need` candidates (larger key first, lower index on ties) and merge
+// both ascending lists into out[0..n_above+need).
+__device__ void finish_row(TopkSmem &sm, const int32_t *alist, uint32_t cnt, uint32_t need, uint32_t n_above,
+                           int32_t *out) {
+    const int tid = threadIdx.x;
+    // choose `need` candidates: larger key first, lower index on ties
+    if (cnt <= (uint32_t)kSmallCand) {
+        // Direct ranking: candidate i is chosen iff fewer than `need`
+        // candidates beat it (larger key, or equal key and lower index).
+        // Candidates sit in index order, so "lower index" is "earlier slot".
+        const int i = tid;
+        const bool act = i < (int)cnt;
+        const uint32_t ki = act ? sm.ckey[i] : 0u;
+        const int32_t ix = act ? sm.cidx[i] : 0;
+        uint32_t rank = 0;
+        for (int j = 0; j < (int)cnt; ++j) {
+            const uint32_t kj = sm.ckey[j];
+            rank += (kj > ki) || (kj == ki && j < i);
+        }
+        const bool chosen = act && rank < need;
+        uint32_t tot;
+        const uint32_t ex = block_scan_packed(chosen ? 1u : 0u, sm.red, &tot);
+        if (chosen) sm.cidx[ex] = ix;  // ex <= i, and slot i was read above
+        __syncthreads();
+    } else {
+        uint32_t T, quota;
+        select_in_candidates(sm, (int)cnt, need, T, quota);
+        uint32_t run_g = 0, run_e = 0;
+        for (int base = 0; base < (int)cnt; base += kThreads) {
+            const int i = base + tid;
+            const uint32_t key = i < (int)cnt ? sm.ckey[i] : 0u;
+            const int32_t ix = i < (int)cnt ? sm.cidx[i] : 0;
+            const bool gt = i < (int)cnt && key > T;
+            const bool eq = i < (int)cnt && key == T;
+            uint32_t tot;
+            const uint32_t ex = block_scan_packed((gt ? 1u : 0u) | (eq ? 0x10000u : 0u), sm.red, &tot);
+            const uint32_t gb = run_g + (ex & 0xFFFFu), eb = run_e + (ex >> 16);
+            // positions only move left and this chunk was read before the scan's barriers
+            if (gt || (eq && eb < quota)) sm.cidx[gb + min(eb, quota)] = ix;
+            run_g += tot & 0xFFFFu;
+            run_e += tot >> 16;
+            __syncthreads();
+        }
+    }
+
+    // ---- merge the two ascending lists into the output
+    const int na = (int)n_above, nd = (int)need;
+    const int32_t *dl = sm.cidx;
+    for (int a = tid; a < na; a += kThreads) {
+        const int32_t v = alist[a];
+        int lo = 0, hi = nd;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (dl[mid] < v) lo = mid + 1; else hi = mid;
+        }
+        out[a + lo] = v;
+    }
+    for (int d = tid; d < nd; d += kThreads) {
+        const int32_t v = dl[d];
+        int lo = 0, hi = na;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (alist[mid] < v) lo = mid + 1; else hi = mid;
+        }
+        out[d + lo] = v;
+    }
+}
+
 __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__restrict__ scores, int64_t ld,
                                                             int row_begin, const int32_t *__restrict__ row_len,
                                                             int max_len, int k, int32_t *__restrict__ idx,
@@ -347,67 +419,207 @@ __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__rest
     }
     __syncthreads();
 
-    // ---- choose `need` candidates: larger key first, lower index on ties
-    if (cnt <= (uint32_t)kSmallCand) {
-        // Direct ranking: candidate i is chosen iff fewer than `need`
-        // candidates beat it (larger key, or equal key and lower index).
-        // Candidates sit in index order, so "lower index" is "earlier slot".
-        const int i = tid;
-        const bool act = i < (int)cnt;
-        const uint32_t ki = act ? sm.ckey[i] : 0u;
-        const int32_t ix = act ? sm.cidx[i] : 0;
-        uint32_t rank = 0;
-        for (int j = 0; j < (int)cnt; ++j) {
-            const uint32_t kj = sm.ckey[j];
-            rank += (kj > ki) || (kj == ki && j < i);
+    finish_row(sm, alist, cnt, need, n_above, out);
+}
+
+
+// ---------------------------------------------------------------------------
+// Long rows, few of them (decode): one thread-block cluster per row.
+//
+// The row is cut into kClusterSize contiguous slices, one per CTA.  Each pass
+// runs on every slice in parallel; the row's value range, the bucket
+// histogram and the per-slice winner / candidate lists are combined through
+// distributed shared memory.  Every exchange is bracketed by hardware cluster
+// barriers (no flag polling), and a CTA leaves only after the last barrier
+// that follows any remote read of its shared memory.  Rank 0 gathers the
+// lists -- slices are in index order, so concatenation keeps the lists
+// ascending -- and finishes the row exactly as the single-CTA kernel does.
+// ---------------------------------------------------------------------------
+
+constexpr int kClusterSize = 8;
+
+struct ClusterExtra {
+    uint32_t ghist[kNB];   // the row's histogram (sum over the cluster)
+    float range[2];        // this slice's min, max
+    uint32_t counts[2];    // this slice's winners, candidates
+};
+
+__host__ __device__ constexpr size_t cluster_smem_bytes(int k) { return smem_bytes(k) + sizeof(ClusterExtra); }
+
+__global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads)
+    topk_rows_cluster_kernel(const float *__restrict__ scores, int64_t ld, int row_begin,
+                             const int32_t *__restrict__ row_len, int max_len, int k, int32_t *__restrict__ idx,
+                             const float *__restrict__ row_stats) {
+    namespace cgs = cooperative_groups;
+    cgs::cluster_group cluster = cgs::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    int32_t *alist = reinterpret_cast<int32_t *>(smem_raw + sizeof(TopkSmem));
+    ClusterExtra &cx = *reinterpret_cast<ClusterExtra *>(smem_raw + smem_bytes(k));
+
+    const int r = blockIdx.x / kClusterSize;
+    const int n = row_length(row_len, r, row_begin, max_len);
+    const float *row = scores + (size_t)r * ld;
+    int32_t *out = idx + (size_t)r * k;
+    const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
+
+    if (n <= k) {  // short row (same decision on every CTA of the cluster)
+        if (rank == 0)
+            for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
+        return;
+    }
+    const int chunk = ((n + kClusterSize - 1) / kClusterSize + 15) / 16 * 16;
+    const int lo = min(n, rank * chunk), m = min(n, lo + chunk) - lo;
+    const float *srow = row + lo;
+
+    // ---- value range of the row
+    float vmin = INFINITY, vmax = -INFINITY;
+    if (row_stats != nullptr) {
+        if (tid < 4) {
+            vmin = __ldg(row_stats + (size_t)r * 8 + 2 * tid);
+            vmax = __ldg(row_stats + (size_t)r * 8 + 2 * tid + 1);
         }
-        const bool chosen = act && rank < need;
-        uint32_t tot;
-        const uint32_t ex = block_scan_packed(chosen ? 1u : 0u, sm.red, &tot);
-        if (chosen) sm.cidx[ex] = ix;  // ex <= i, and slot i was read above
-        __syncthreads();
     } else {
-        uint32_t T, quota;
-        select_in_candidates(sm, (int)cnt, need, T, quota);
-        uint32_t run_g = 0, run_e = 0;
-        for (int base = 0; base < (int)cnt; base += kThreads) {
-            const int i = base + tid;
-            const uint32_t key = i < (int)cnt ? sm.ckey[i] : 0u;
-            const int32_t ix = i < (int)cnt ? sm.cidx[i] : 0;
-            const bool gt = i < (int)cnt && key > T;
-            const bool eq = i < (int)cnt && key == T;
-            uint32_t tot;
-            const uint32_t ex = block_scan_packed((gt ? 1u : 0u) | (eq ? 0x10000u : 0u), sm.red, &tot);
-            const uint32_t gb = run_g + (ex & 0xFFFFu), eb = run_e + (ex >> 16);
-            // positions only move left and this chunk was read before the scan's barriers
-            if (gt || (eq && eb < quota)) sm.cidx[gb + min(eb, quota)] = ix;
-            run_g += tot & 0xFFFFu;
-            run_e += tot >> 16;
-            __syncthreads();
+        for (int i0 = tid * kVec; i0 < m; i0 += kChunk) {
+            float x[kVec];
+            const int c = load_vals(srow, i0, m, x);
+#pragma unroll
+            for (int j = 0; j < kVec; ++j)
+                if (j < c) {
+                    vmin = fminf(vmin, x[j]);
+                    vmax = fmaxf(vmax, x[j]);
+                }
         }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        vmin = fminf(vmin, __shfl_xor_sync(0xFFFFFFFFu, vmin, o));
+        vmax = fmaxf(vmax, __shfl_xor_sync(0xFFFFFFFFu, vmax, o));
+    }
+    float *fred = reinterpret_cast<float *>(sm.red);
+    if (lane == 0) {
+        fred[warp] = vmin;
+        fred[kWarps + warp] = vmax;
+    }
+    for (int i = tid; i < kNB; i += kThreads) sm.hist[i] = 0;
+    __syncthreads();
+    if (tid == 0) {
+        float a = fred[0], b = fred[kWarps];
+        for (int w = 1; w < kWarps; ++w) {
+            a = fminf(a, fred[w]);
+            b = fmaxf(b, fred[kWarps + w]);
+        }
+        cx.range[0] = a;
+        cx.range[1] = b;
+    }
+    cluster.sync();
+    vmin = INFINITY;
+    vmax = -INFINITY;
+    for (int q = 0; q < kClusterSize; ++q) {
+        const float *rr = cluster.map_shared_rank(cx.range, q);
+        vmin = fminf(vmin, rr[0]);
+        vmax = fmaxf(vmax, rr[1]);
+    }
+    cluster.sync();  // every remote read of the ranges is done
+    if (vmin == vmax) {  // every entry ties: the k lowest indices
+        if (rank == 0)
+            for (int i = tid; i < k; i += kThreads) out[i] = i;
+        return;
+    }
+    const float range = vmax - vmin;
+    if (!(range < INFINITY)) {
+        if (rank == 0) topk_row_radix(row, n, k, out, sm);
+        return;
+    }
+    const float scale = __fdiv_rn((float)kNB * 0.99999f, range);
+
+    // ---- histogram of this slice, then of the row
+    for (int i0 = tid * kVec; i0 < m; i0 += kChunk) {
+        float x[kVec];
+        const int c = load_vals(srow, i0, m, x);
+#pragma unroll
+        for (int j = 0; j < kVec; ++j)
+            if (j < c) atomicAdd(&sm.hist[bucket_of(x[j], vmin, scale)], 1u);
+    }
+    __syncthreads();
+    cluster.sync();
+    for (int b = tid; b < kNB; b += kThreads) {
+        uint32_t sum = 0;
+        for (int q = 0; q < kClusterSize; ++q) sum += cluster.map_shared_rank(sm.hist, q)[b];
+        cx.ghist[b] = sum;
+    }
+    __syncthreads();
+    find_threshold_bin(cx.ghist, (uint32_t)k, sm.red, sm.bcast);
+    const uint32_t Bt = sm.bcast[0];
+    const uint32_t need = sm.bcast[1];
+    const uint32_t n_above = sm.bcast[2];
+    const uint32_t cnt = cx.ghist[Bt];
+    cluster.sync();  // every remote read of the histograms is done
+    if (cnt > (uint32_t)kCap) {
+        if (rank == 0) topk_row_radix(row, n, k, out, sm);
+        return;
     }
 
-    // ---- merge the two ascending lists into the output
-    const int na = (int)n_above, nd = (int)need;
-    const int32_t *dl = sm.cidx;
-    for (int a = tid; a < na; a += kThreads) {
-        const int32_t v = alist[a];
-        int lo = 0, hi = nd;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (dl[mid] < v) lo = mid + 1; else hi = mid;
+    // ---- ordered collect of this slice
+    uint32_t run_a = 0, run_c = 0;
+    for (int base = 0; base < m; base += kChunk) {
+        const int i0 = base + tid * kVec;
+        float x[kVec] = {};
+        const int c = i0 < m ? load_vals(srow, i0, m, x) : 0;
+        uint32_t cls[kVec];
+        uint32_t na = 0, nc = 0;
+#pragma unroll
+        for (int j = 0; j < kVec; ++j) {
+            const uint32_t b = bucket_of(x[j], vmin, scale);
+            cls[j] = j >= c ? 0u : (b > Bt ? 2u : (b == Bt ? 1u : 0u));
+            na += cls[j] == 2u;
+            nc += cls[j] == 1u;
         }
-        out[a + lo] = v;
-    }
-    for (int d = tid; d < nd; d += kThreads) {
-        const int32_t v = dl[d];
-        int lo = 0, hi = na;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (alist[mid] < v) lo = mid + 1; else hi = mid;
+        uint32_t tot;
+        const uint32_t ex = block_scan_packed(na | (nc << 16), sm.red, &tot);
+        uint32_t pa = run_a + (ex & 0xFFFFu), pc = run_c + (ex >> 16);
+#pragma unroll
+        for (int j = 0; j < kVec; ++j) {
+            if (cls[j] == 2u) alist[pa++] = lo + i0 + j;
+            if (cls[j] == 1u) {
+                sm.ckey[pc] = order_key(x[j]);
+                sm.cidx[pc] = lo + i0 + j;
+                ++pc;
+            }
         }
-        out[d + lo] = v;
+        run_a += tot & 0xFFFFu;
+        run_c += tot >> 16;
     }
+    if (tid == 0) {
+        cx.counts[0] = run_a;
+        cx.counts[1] = run_c;
+    }
+    __syncthreads();
+    cluster.sync();
+
+    // ---- rank 0 appends the other slices' lists (in rank = index order)
+    if (rank == 0) {
+        uint32_t off_a = run_a, off_c = run_c;
+        for (int q = 1; q < kClusterSize; ++q) {
+            const uint32_t *qc = cluster.map_shared_rank(cx.counts, q);
+            const uint32_t qa = qc[0], qn = qc[1];
+            const int32_t *qal = reinterpret_cast<const int32_t *>(
+                reinterpret_cast<const uint8_t *>(cluster.map_shared_rank(&sm, q)) + sizeof(TopkSmem));
+            const TopkSmem *qs = cluster.map_shared_rank(&sm, q);
+            for (uint32_t i = tid; i < qa; i += kThreads) alist[off_a + i] = qal[i];
+            for (uint32_t i = tid; i < qn; i += kThreads) {
+                sm.ckey[off_c + i] = qs->ckey[i];
+                sm.cidx[off_c + i] = qs->cidx[i];
+            }
+            off_a += qa;
+            off_c += qn;
+        }
+        __syncthreads();
+    }
+    cluster.sync();  // rank 0 has read every remote list
+    if (rank != 0) return;
+    finish_row(sm, alist, cnt, need, n_above, out);
 }
 
 }  // namespace
@@ -418,6 +630,20 @@ cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_ro
                         int max_len, int k, int32_t *idx, const float *row_stats, void *, size_t,
                         cudaStream_t stream) {
     if (n_rows == 0) return cudaSuccess;
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (max_len >= 16384 && n_rows < (sms > 0 ? sms : 148)) {
+        // few long rows: a cluster of CTAs per row keeps every SM busy
+        const size_t csmem = cluster_smem_bytes(k);
+        if (csmem > 220 * 1024) return cudaErrorInvalidValue;
+        cudaError_t e = cudaFuncSetAttribute(topk_rows_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)csmem);
+        if (e != cudaSuccess) return e;
+        topk_rows_cluster_kernel<<<n_rows * kClusterSize, kThreads, csmem, stream>>>(scores, ld, row_begin, row_len,
+                                                                                       max_len, k, idx, row_stats);
+        return cudaGetLastError();
+    }
     const size_t smem = smem_bytes(k);
     if (smem > 220 * 1024) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -427,6 +653,6 @@ cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_ro
     return cudaGetLastError();
 }
 
-bool topk_k_supported(int k) { return smem_bytes(k) <= 220 * 1024; }
+bool topk_k_supported(int k) { return cluster_smem_bytes(k) <= 220 * 1024; }
 
 }  // namespace dsa
