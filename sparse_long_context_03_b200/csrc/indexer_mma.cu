@@ -138,25 +138,39 @@ __global__ void __launch_bounds__(256) indexer_prefill_mma_kernel(
     }
 }
 
-constexpr int kDecodePagesPerCta = 8;  // one page (64 keys) per warp
+constexpr int kDecodeWarps = 8;
+constexpr int kDecodePagesPerWarp = 4;
+constexpr int kDecodePagesPerCta = kDecodeWarps * kDecodePagesPerWarp;
+
+// Shared staging of one cached page: 64 key rows at a pitch of dI + 16 bytes
+// (8 rows read by one ldmatrix then start in 8 different bank groups), then
+// the 64 key scales.
+template <int DI>
+constexpr int page_stage_bytes() {
+    return kPage * (DI + 16) + kPage * 4;
+}
 
 template <int DI, int NT>
-__global__ void __launch_bounds__(256, 2) indexer_decode_mma_kernel(
+__global__ void __launch_bounds__(kDecodeWarps * 32, 2) indexer_decode_mma_kernel(
     const uint8_t *__restrict__ q8, const float *__restrict__ sq, const float *__restrict__ w,
     const uint8_t *__restrict__ k8c, const float *__restrict__ skc, const int32_t *__restrict__ block_table,
     int max_pages, int num_pages, const int32_t *__restrict__ seq_lens, int max_seq_len, int HI,
     float *__restrict__ scores, int64_t ld) {
     constexpr int KS = DI / 32;
+    constexpr int PITCH = DI + 16;
+    constexpr int STAGE = page_stage_bytes<DI>();
+    constexpr int CPR = DI / 16;  // 16-byte chunks per key row
+    extern __shared__ __align__(16) uint8_t smem[];
     const int b = blockIdx.y;
     const int n = min(min(__ldg(seq_lens + b), max_seq_len), max_pages * kPage);
     const int warp = threadIdx.x >> 5, lane = lane_id(), gid = lane >> 2, tig = lane & 3;
-    const int lp = blockIdx.x * kDecodePagesPerCta + warp;   // logical page of this warp
-    const int sb = lp * kPage;
-    if (sb >= n) return;
+    const int lp0 = blockIdx.x * kDecodePagesPerCta + warp;   // this warp's pages: lp0 + kDecodeWarps * i
+    if (lp0 * kPage >= n) return;
+    uint8_t *ws = smem + warp * 2 * STAGE;
+    const uint32_t ws_u32 = smem_u32(ws);
 
     // Query fragments (m16n8k32 B operand, column n = head): b0 bytes
-    // ks*32 + tig*4 of head nt*8+gid, b1 the same +16.  Loaded once, used for
-    // the page's four 16-key tiles.
+    // ks*32 + tig*4 of head nt*8+gid, b1 the same +16.
     uint32_t qf[NT][KS][2];
     float wf[NT][2];
 #pragma unroll
@@ -175,33 +189,58 @@ __global__ void __launch_bounds__(256, 2) indexer_decode_mma_kernel(
         }
     }
     const float f = __ldg(sq + b);
-    const int page = __ldg(block_table + (size_t)b * max_pages + lp);
-    const bool page_ok = page >= 0 && page < num_pages;
-    const uint8_t *pk = k8c + (size_t)(page_ok ? page : 0) * kPage * DI;
-    const float *ps = skc + (size_t)(page_ok ? page : 0) * kPage;
     float *srow = scores + (size_t)b * ld;
 
-    // all four tiles' key fragments in flight at once
-    uint32_t a[4][KS][4];
-    float skv[4][2];
+    auto page_of = [&](int i) -> int { return lp0 + kDecodeWarps * i; };
+    auto page_id = [&](int lp) -> int {
+        const int pg = __ldg(block_table + (size_t)b * max_pages + lp);
+        return (pg >= 0 && pg < num_pages) ? pg : -1;
+    };
+    auto issue = [&](int i) {
+        const int lp = page_of(i);
+        const int pg = page_id(lp);
+        const uint32_t st = ws_u32 + (uint32_t)((i & 1) * STAGE);
+        const uint8_t *src = k8c + (size_t)(pg < 0 ? 0 : pg) * kPage * DI;
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const int k0 = m * 16 + gid, k8 = k0 + 8;
-        load_key_frags<DI>(a[m], pk + (size_t)k0 * DI, pk + (size_t)k8 * DI, page_ok && sb + k0 < n,
-                           page_ok && sb + k8 < n, tig);
-        skv[m][0] = (page_ok && sb + k0 < n) ? __ldg(ps + k0) : 0.f;
-        skv[m][1] = (page_ok && sb + k8 < n) ? __ldg(ps + k8) : 0.f;
-    }
+        for (int c = lane; c < kPage * CPR; c += 32) {
+            const int row = c / CPR, ch = c % CPR;
+            cp_async_16(st + row * PITCH + ch * 16, src + row * DI + ch * 16);
+        }
+        if (lane < kPage * 4 / 16) cp_async_16(st + kPage * PITCH + lane * 16,
+                                                skc + (size_t)(pg < 0 ? 0 : pg) * kPage + lane * 4);
+    };
+    int np = 0;
+    while (np < kDecodePagesPerWarp && page_of(np) * kPage < n) ++np;
+    issue(0);
+    cp_async_commit();
+    for (int i = 0; i < np; ++i) {
+        if (i + 1 < np) issue(i + 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncwarp();
+        const int lp = page_of(i);
+        const bool page_ok = page_id(lp) >= 0;
+        const int sb = lp * kPage;
+        const uint32_t st = ws_u32 + (uint32_t)((i & 1) * STAGE);
+        const float *sks = reinterpret_cast<const float *>(ws + (i & 1) * STAGE + kPage * PITCH);
+#pragma unroll 1
+        for (int m = 0; m < 4; ++m) {
+            uint32_t a[KS][4];
+            const int row = m * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        float p0, p1;
-        score_16keys<KS, NT>(
-            a[m], [&](int nt, int ks, int half) { return qf[nt][ks][half]; },
-            [&](int nt, int i) { return wf[nt][i]; }, p0, p1);
-        const int key0 = sb + m * 16 + gid, key8 = key0 + 8;
-        if (tig == 0 && key0 < n) srow[key0] = page_ok ? p0 * f * skv[m][0] : -INFINITY;
-        if (tig == 1 && key8 < n) srow[key8] = page_ok ? p1 * f * skv[m][1] : -INFINITY;
+            for (int ks = 0; ks < KS; ++ks) ldmatrix_x4(a[ks], st + row * PITCH + ks * 32 + (lane >> 4) * 16);
+            float p0, p1;
+            score_16keys<KS, NT>(
+                a, [&](int nt, int ks, int half) { return qf[nt][ks][half]; },
+                [&](int nt, int j) { return wf[nt][j]; }, p0, p1);
+            const int k0 = m * 16 + gid, k8 = k0 + 8;
+            const int key0 = sb + k0, key8 = sb + k8;
+            if (tig == 0 && key0 < n) srow[key0] = page_ok ? p0 * f * sks[k0] : -INFINITY;
+            if (tig == 1 && key8 < n) srow[key8] = page_ok ? p1 * f * sks[k8] : -INFINITY;
+        }
+        __syncwarp();
     }
+    cp_async_wait<0>();
 }
 
 // Calls launch(integral_constant<DI>, integral_constant<NT>) for a supported
@@ -285,13 +324,19 @@ cudaError_t launch_indexer_decode(const uint8_t *q8, const float *sq, const floa
     if (B == 0 || max_seq_len == 0) return cudaSuccess;
     const int pages = (max_seq_len + kPage - 1) / kPage;
     const dim3 grid((pages + kDecodePagesPerCta - 1) / kDecodePagesPerCta, B);
+    cudaError_t err = cudaSuccess;
     const bool ok = dispatch_shape(HI, dI, [&](auto di, auto nt) {
         constexpr int DI = decltype(di)::value, NT = decltype(nt)::value;
-        indexer_decode_mma_kernel<DI, NT><<<grid, 256, 0, stream>>>(
+        constexpr int smem = kDecodeWarps * 2 * page_stage_bytes<DI>();
+        err = cudaFuncSetAttribute(indexer_decode_mma_kernel<DI, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   smem);
+        if (err != cudaSuccess) return true;
+        indexer_decode_mma_kernel<DI, NT><<<grid, kDecodeWarps * 32, smem, stream>>>(
             q8, sq, w, k8c, skc, block_table, max_pages, num_pages, seq_lens, max_seq_len, HI, scores, ld);
+        err = cudaGetLastError();
         return true;
     });
-    return ok ? cudaGetLastError() : cudaErrorInvalidValue;
+    return ok ? err : cudaErrorInvalidValue;
 }
 
 }  // namespace dsa
