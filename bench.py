@@ -221,6 +221,7 @@ def run_prefill_timed(pb, steps, warmup, world, gpu_index):
         end.record(pb.stream)
         torch.cuda.synchronize()
     barrier(world)
+    pb.dsa.check_device_error()  # a kernel that gave up a bounded wait voids the run
     ms = start.elapsed_time(end)
     per = {}
     for name, lst in ev.items():
@@ -256,6 +257,7 @@ def run_prefill_e2e(pb, steps, warmup):
         one()
     e.record(pb.stream)
     torch.cuda.synchronize()
+    dsa.check_device_error()
     ms = s.elapsed_time(e)
     del dev, host
     return ms, h2d, d2h
@@ -303,6 +305,7 @@ def run_decode_timed(db, steps, warmup):
         db.step()
     e.record(db.stream)
     torch.cuda.synchronize()
+    db.dsa.check_device_error()
     return s.elapsed_time(e) / steps
 
 

@@ -172,8 +172,8 @@ DSA_API dsa_status_t dsa_sparse_gqa_prefill(const uint16_t *Q, const uint16_t *K
  *   idx_out       [B, k] int32 selected indices, may be NULL
  *   ws            >= dsa_decode_workspace_size(...) bytes
  * A token on a page id outside [0, num_pages) scores -inf and is skipped by
- * the attention.  k8_cache and k_scale_cache start on 16-byte boundaries
- * (DSA_ERR_INVALID_ARG otherwise): pages are copied in 16-byte pieces.
+ * the attention.  q8, k8_cache and k_scale_cache start on 16-byte boundaries
+ * (DSA_ERR_INVALID_ARG otherwise): they are copied in 16-byte pieces.
  * dsa_sparse_gqa_decode runs the three stages below on `stream`:
  * scores (dsa_decode_indexer_scores) -> top-k (dsa_topk with row_len =
  * seq_lens) -> attention (dsa_sparse_gqa_decode_attention).

@@ -66,8 +66,8 @@ def _load():
         lib.dsa_oracle_indexer.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I64]
         lib.dsa_oracle_topk.argtypes = [P, I64, P, I, I, P]
         lib.dsa_oracle_sparse_attention.argtypes = [P, P, P, P, I, I, I, I, I, I, D, P, P]
-        lib.dsa_oracle_decode_indexer.argtypes = [P, P, P, P, P, P, I, I, P, I, I, I, P, I64]
-        lib.dsa_oracle_decode_attention.argtypes = [P, P, P, P, I, I, P, P, I, I, I, I, I, D, P, P]
+        lib.dsa_oracle_decode_indexer.argtypes = [P, P, P, P, P, P, I, I, I, P, I, I, I, P, I64]
+        lib.dsa_oracle_decode_attention.argtypes = [P, P, P, P, I, I, I, P, P, I, I, I, I, I, D, P, P]
         for f in ("dsa_oracle_indexer", "dsa_oracle_topk", "dsa_oracle_sparse_attention",
                   "dsa_oracle_decode_indexer", "dsa_oracle_decode_attention"):
             getattr(lib, f).restype = I
@@ -174,7 +174,8 @@ def sparse_attention(Q, K, V, idx, row_begin: int, sm_scale: float):
 
 
 def decode_indexer(q8, sq, w, k8_cache, sk_cache, block_table, seq_lens, ld: int | None = None):
-    """Paged decode indexer; returns float64 [B, ld], -inf past each seq_len."""
+    """Paged decode indexer; returns float64 [B, ld], -inf past each seq_len
+    and for tokens whose page id is not a page of the cache."""
     q8 = _c(q8, np.uint8)
     sq = _c(sq, np.float32)
     w = _c(w, np.float32)
@@ -189,7 +190,8 @@ def decode_indexer(q8, sq, w, k8_cache, sk_cache, block_table, seq_lens, ld: int
         ld = int(seq_lens.max()) if B else 1
     out = np.empty((B, ld), np.float64)
     _check(_load().dsa_oracle_decode_indexer(_p(q8), _p(sq), _p(w), _p(k8_cache), _p(sk_cache),
-                                             _p(block_table), max_pages, page, _p(seq_lens), B, HI, dI,
+                                             _p(block_table), max_pages, page, k8_cache.shape[0], _p(seq_lens),
+                                             B, HI, dI,
                                              _p(out), ld), "decode_indexer")
     return out
 
@@ -209,7 +211,7 @@ def decode_attention(q, k_cache, v_cache, block_table, seq_lens, idx, sm_scale: 
     out = np.empty((B, Hq, D), np.float64)
     lse = np.empty((B, Hq), np.float64)
     _check(_load().dsa_oracle_decode_attention(_p(q), _p(k_cache), _p(v_cache), _p(block_table), max_pages,
-                                               page, _p(seq_lens), _p(idx), B, Hq, Hkv, D, k,
+                                               page, k_cache.shape[0], _p(seq_lens), _p(idx), B, Hq, Hkv, D, k,
                                                float(sm_scale), _p(out), _p(lse)), "decode_attention")
     return out, lse
 

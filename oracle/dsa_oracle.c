@@ -279,11 +279,11 @@ EXPORT int dsa_oracle_sparse_attention(const uint16_t *Q, const uint16_t *K, con
  * k8_cache [P,page,dI], sk_cache [P,page]; out[b*ld + s], -inf past seq_len. */
 EXPORT int dsa_oracle_decode_indexer(const uint8_t *q8, const float *sq, const float *w,
                                      const uint8_t *k8_cache, const float *sk_cache,
-                                     const int32_t *block_table, int max_pages, int page,
+                                     const int32_t *block_table, int max_pages, int page, int num_pages,
                                      const int32_t *seq_lens, int B, int HI, int dI,
                                      double *out, int64_t ld)
 {
-    if (B < 0 || HI < 1 || dI < 1 || page < 1 || max_pages < 1) return -1;
+    if (B < 0 || HI < 1 || dI < 1 || page < 1 || max_pages < 1 || num_pages < 1) return -1;
     for (int b = 0; b < B; ++b)
         if (seq_lens[b] < 0 || seq_lens[b] > ld || seq_lens[b] > (int64_t)max_pages * page) return -1;
 #pragma omp parallel for schedule(dynamic, 1)
@@ -291,6 +291,9 @@ EXPORT int dsa_oracle_decode_indexer(const uint8_t *q8, const float *sq, const f
         for (int64_t s = 0; s < ld; ++s) {
             if (s >= seq_lens[b]) { out[(size_t)b * ld + s] = -INFINITY; continue; }
             int32_t p = block_table[(size_t)b * max_pages + s / page];
+            /* library convention (not from the papers): a token whose page id
+             * is not a cache page has no key and scores -inf */
+            if (p < 0 || p >= num_pages) { out[(size_t)b * ld + s] = -INFINITY; continue; }
             size_t slot = (size_t)p * page + (size_t)(s % page);
             out[(size_t)b * ld + s] = indexer_pair(q8 + (size_t)b * HI * dI, sq[b], w + (size_t)b * HI,
                                                    k8_cache + slot * dI, sk_cache[slot], HI, dI);
@@ -301,14 +304,15 @@ EXPORT int dsa_oracle_decode_indexer(const uint8_t *q8, const float *sq, const f
 
 /* Attention for one query per sequence over the selected cached rows.
  * q [B,Hq,D]; k_cache, v_cache [P,page,Hkv,D]; idx [B,k] (entries outside
- * [0, seq_len) are ignored); out [B,Hq,D]; lse nullable [B,Hq]. */
+ * [0, seq_len) or on a page id outside [0, num_pages) are ignored);
+ * out [B,Hq,D]; lse nullable [B,Hq]. */
 EXPORT int dsa_oracle_decode_attention(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
-                                       const int32_t *block_table, int max_pages, int page,
+                                       const int32_t *block_table, int max_pages, int page, int num_pages,
                                        const int32_t *seq_lens, const int32_t *idx,
                                        int B, int Hq, int Hkv, int D, int k, double sm_scale,
                                        double *out, double *lse)
 {
-    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || D < 1 || k < 1 || page < 1) return -1;
+    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || D < 1 || k < 1 || page < 1 || num_pages < 1) return -1;
     int G = Hq / Hkv;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int b = 0; b < B; ++b) {
@@ -321,6 +325,7 @@ EXPORT int dsa_oracle_decode_attention(const uint16_t *q, const uint16_t *k_cach
                 int32_t s = idx[(size_t)b * k + i];
                 if (s < 0 || s >= seq_lens[b]) continue;
                 int32_t p = block_table[(size_t)b * max_pages + s / page];
+                if (p < 0 || p >= num_pages) continue; /* unmapped page: no key, skipped */
                 size_t slot = (size_t)p * page + (size_t)(s % page);
                 kr[n] = k_cache + (slot * Hkv + g) * D;
                 vr[n] = v_cache + (slot * Hkv + g) * D;

@@ -121,9 +121,10 @@ dsa_status_t dsa_sparse_gqa_prefill(const uint16_t *Q, const uint16_t *K, const 
                                                   as_stream(stream)));
 }
 
-// The decode indexer copies cache pages with 16-byte cp.async.
-static bool paged_keys_aligned(const uint8_t *k8_cache, const float *k_scale_cache) {
-    return (reinterpret_cast<uintptr_t>(k8_cache) | reinterpret_cast<uintptr_t>(k_scale_cache)) % 16 == 0;
+// The decode indexer copies cache pages and query rows in 16-byte pieces.
+static bool paged_keys_aligned(const uint8_t *q8, const uint8_t *k8_cache, const float *k_scale_cache) {
+    return (reinterpret_cast<uintptr_t>(q8) | reinterpret_cast<uintptr_t>(k8_cache) |
+            reinterpret_cast<uintptr_t>(k_scale_cache)) % 16 == 0;
 }
 
 static dsa_status_t check_decode_common(const int32_t *block_table, int max_pages, int num_pages,
@@ -144,7 +145,7 @@ dsa_status_t dsa_decode_indexer_scores(const uint8_t *q8, const float *q_scale, 
     if (!dsa::indexer_shape_supported(HI, dI)) return DSA_ERR_UNSUPPORTED_SHAPE;
     if (B == 0 || max_seq_len == 0) return DSA_OK;
     if (!q8 || !q_scale || !w || !k8_cache || !k_scale_cache || !scores) return DSA_ERR_INVALID_ARG;
-    if (!paged_keys_aligned(k8_cache, k_scale_cache)) return DSA_ERR_INVALID_ARG;
+    if (!paged_keys_aligned(q8, k8_cache, k_scale_cache)) return DSA_ERR_INVALID_ARG;
     if (ld_scores < max_seq_len || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
     return cuda_status(dsa::launch_indexer_decode(q8, q_scale, w, k8_cache, k_scale_cache, block_table, max_pages,
                                                   num_pages, seq_lens, max_seq_len, B, HI, dI, scores, ld_scores,
@@ -214,7 +215,7 @@ dsa_status_t dsa_sparse_gqa_decode(const uint16_t *q, const uint8_t *q8, const f
     if (B == 0) return DSA_OK;
     if (!q || !q8 || !q_scale || !w || !k8_cache || !k_scale_cache || !k_cache || !v_cache || !out)
         return DSA_ERR_INVALID_ARG;
-    if (!paged_keys_aligned(k8_cache, k_scale_cache)) return DSA_ERR_INVALID_ARG;
+    if (!paged_keys_aligned(q8, k8_cache, k_scale_cache)) return DSA_ERR_INVALID_ARG;
     const DecodeWs L = decode_ws_layout(B, max_seq_len, Hq, Hkv, D, k);
     if (ws == nullptr || ws_bytes < L.total) return DSA_ERR_WORKSPACE;
     char *base = static_cast<char *>(ws);

@@ -322,6 +322,10 @@ cudaError_t launch_indexer_decode(const uint8_t *q8, const float *sq, const floa
                                   const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI, float *scores,
                                   int64_t ld, cudaStream_t stream) {
     if (B == 0 || max_seq_len == 0) return cudaSuccess;
+    // tensor-core path; this one serves batches beyond its shared-memory prefix
+    if (indexer_decode_tc_supported(HI, dI, B, max_seq_len))
+        return launch_indexer_decode_tc(q8, sq, w, k8c, skc, block_table, max_pages, num_pages, seq_lens, max_seq_len,
+                                        B, HI, dI, scores, ld, stream);
     const int pages = (max_seq_len + kPage - 1) / kPage;
     const dim3 grid((pages + kDecodePagesPerCta - 1) / kDecodePagesPerCta, B);
     cudaError_t err = cudaSuccess;

@@ -350,6 +350,413 @@ __global__ void __launch_bounds__(EpiShape<HI>::kThreads, 1) indexer_tc_kernel(c
     }
 }
 
+// ===========================================================================
+// Decode: one query token per sequence against its paged cache ("Kwai
+// Keye-VL-2.0 Technical Report" review, DSA decode, section 5.3).
+//
+// GEMM view: A = 128 cached keys, i.e. two 64-token pages (K-major rows of
+// dI bytes, one TMA box per page), B = the sequence's HI indexer heads padded
+// to N = max(16, HI) rows, D = 128 x N fp32 in TMEM (lane = key, column =
+// head).  A step is up to SP pages of one sequence (SP = 8 for dI <= 64, 4 for
+// dI = 128): SP/2 such tiles into SP/2 accumulators.  A sequence of n tokens
+// has ceil(n / (64 SP)) steps; the steps of the whole batch are numbered
+// through a prefix sum over the sequences and split into equal contiguous
+// ranges, one per CTA, so long and short sequences share the SMs evenly.
+//
+// Warp roles (one CTA per SM):
+//   producers  four warps share every step: warp p issues the TMA boxes of
+//              pages 2p and 2p+1 (SP = 8) plus bulk copies of their 64 key
+//              scales.  One thread issuing bulk copies moves about a third of
+//              what the SM's HBM share needs; four of them reach it.  Each
+//              warp looks up the page ids of 32 consecutive steps at a time.
+//              The first producer also writes the step's 16-byte record
+//              (sequence, step, length, page validity) and copies each
+//              sequence's query rows, in sequence order, into one of two
+//              swizzled query slots;
+//   MMA        (SP/2) x (dI/32) UMMAs per step into an (SP/2) x N column
+//              accumulator.  Its fixed cost per step (barrier waits, fences,
+//              commits: several hundred cycles) is what sizes the step;
+//   epilogue   kDecGroups groups of four warps take alternate steps: per tile
+//              each thread owns one key, reads its N columns, ReLU and the
+//              head-weighted sum, the two scales, and stores one score.
+// A stage is refilled once its UMMAs completed and the epilogue group read
+// its scales and record (five arrivals).
+// ===========================================================================
+
+constexpr int kDecMaxB = 4096;     // sequences whose step prefix fits in shared memory
+constexpr int kDecPage = 64;       // tokens per cache page
+constexpr int kDecGroups = 2;
+constexpr int kDecProducers = 4;
+constexpr int kDecProducer0 = 4 * kDecGroups;         // warps 0 .. 4G-1: epilogue
+constexpr int kDecMmaWarp = kDecProducer0 + kDecProducers;
+constexpr int kDecThreads = (kDecMmaWarp + 1) * 32;
+// 13 warps leave four on one scheduler, whose 16K registers cap a thread at 128.
+constexpr int kDecMaxRegs = 128;
+
+template <int N, int DI>
+struct DecLayout {
+    static constexpr int SP = DI > 64 ? 4 : 8;                   // pages per step
+    static constexpr int kTiles = SP / 2;                        // 128-key MMA tiles per step
+    static constexpr int kKeyBytes = SP * kDecPage * DI;
+    static constexpr int kScales = kKeyBytes;                    // SP * 64 floats
+    static constexpr int kMeta = kScales + SP * kDecPage * 4;    // int4 record
+    static constexpr int kStageBytes = (kMeta + 16 + 1023) / 1024 * 1024;
+    static constexpr int kQBytes = (N * DI + 1023) / 1024 * 1024;
+    static constexpr int kPrefixBytes = ((kDecMaxB + 1) * 4 + 15) / 16 * 16;
+    static constexpr int kFixed = 2 * kQBytes + kPrefixBytes + 1024;
+    static constexpr int kStages = (212 * 1024 - kFixed) / kStageBytes;
+    static constexpr int kAccCols = kTiles * N;                  // TMEM columns per step
+    static constexpr int kAccBufs = 512 / kAccCols > 8 ? 8 : 512 / kAccCols;
+    static constexpr int kQ = kStages * kStageBytes;
+    static constexpr int kPrefix = kQ + 2 * kQBytes;
+    static constexpr int kBars = kPrefix + kPrefixBytes;
+    static constexpr int kNumBars = 2 * kStages + 4 + 2 * kAccBufs + 1;
+    static constexpr int kTmemSlot = kBars + kNumBars * 8;
+    static constexpr int kBytes = kTmemSlot + 16;
+    static constexpr int kAlloc = kBytes + 1024;
+    static_assert(SP == 2 * kDecProducers || SP == kDecProducers, "pages per producer");
+    static_assert(kStages >= 4, "decode indexer ring too shallow");
+    static_assert(kAccBufs % kDecGroups == 0, "an accumulator serves one epilogue group");
+    static_assert(kAlloc <= 227 * 1024, "decode indexer shared memory");
+};
+
+// In-place inclusive prefix sum of a[0..n) by the whole block; `scratch`
+// holds blockDim.x ints.
+__device__ void block_inclusive_scan(int *a, int n, int *scratch) {
+    const int T = blockDim.x, t = threadIdx.x;
+    const int chunk = (n + T - 1) / T;
+    const int lo = min(n, t * chunk), hi = min(n, lo + chunk);
+    int sum = 0;
+    for (int i = lo; i < hi; ++i) sum += a[i];
+    scratch[t] = sum;
+    __syncthreads();
+    if (t < 32) {
+        int carry = 0;
+        for (int base = 0; base < T; base += 32) {
+            const int v = base + t < T ? scratch[base + t] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (t >= o) incl += u;
+            }
+            if (base + t < T) scratch[base + t] = carry + incl - v;
+            carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+    }
+    __syncthreads();
+    int run = scratch[t];
+    for (int i = lo; i < hi; ++i) {
+        run += a[i];
+        a[i] = run;
+    }
+    __syncthreads();
+}
+
+template <int N, int DI>
+__global__ void __maxnreg__(kDecMaxRegs) indexer_decode_tc_kernel(
+    const __grid_constant__ CUtensorMap tmap_k, const uint8_t *__restrict__ q8, const float *__restrict__ sq,
+    const float *__restrict__ w, const float *__restrict__ skc, const int32_t *__restrict__ block_table,
+    int max_pages, int num_pages, const int32_t *__restrict__ seq_lens, int max_seq_len, int B, int HI,
+    float *__restrict__ scores, int64_t ld) {
+    using Lay = DecLayout<N, DI>;
+    constexpr int S = Lay::kStages, A = Lay::kAccBufs, G = kDecGroups;
+    constexpr int SP = Lay::SP, T = Lay::kTiles, PPW = SP / kDecProducers;  // pages per producer warp
+    constexpr int KSTEPS = DI / 32;
+    constexpr int CPR = DI / 16;  // 16-byte chunks per key or query row
+    constexpr uint32_t IDESC = tc::idesc_e4m3_f32(2 * kDecPage, N);
+    constexpr uint32_t kPageTx = kDecPage * DI + kDecPage * 4;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    int *prefix = reinterpret_cast<int *>(smem + Lay::kPrefix);
+    const uint32_t bars = sbase + Lay::kBars;
+    auto full_bar = [&](int s) { return bars + 8u * s; };
+    auto empty_bar = [&](int s) { return bars + 8u * (S + s); };
+    auto qfull_bar = [&](int q) { return bars + 8u * (2 * S + q); };
+    auto qempty_bar = [&](int q) { return bars + 8u * (2 * S + 2 + q); };
+    auto tfull_bar = [&](int a) { return bars + 8u * (2 * S + 4 + a); };
+    auto tempty_bar = [&](int a) { return bars + 8u * (2 * S + 4 + A + a); };
+    const uint32_t mma_done_bar = bars + 8u * (2 * S + 4 + 2 * A);
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + Lay::kTmemSlot);
+
+    const int warp = threadIdx.x >> 5, lane = lane_id();
+    const int cap = min(max_seq_len, max_pages * kDecPage);
+    auto seq_len_of = [&](int b) { return min(max(__ldg(seq_lens + b), 0), cap); };
+
+    // steps per sequence, then their prefix: prefix[b] = first step of b
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+        const int pages = (seq_len_of(b) + kDecPage - 1) / kDecPage;
+        prefix[b + 1] = (pages + SP - 1) / SP;
+    }
+    if (threadIdx.x == 0) {
+        prefix[0] = 0;
+        for (int s = 0; s < S; ++s) {
+            tc::mbar_init(full_bar(s), kDecProducers);
+            tc::mbar_init(empty_bar(s), 1 + 4);
+        }
+        for (int q = 0; q < 2; ++q) {
+            tc::mbar_init(qfull_bar(q), 1);
+            tc::mbar_init(qempty_bar(q), 1);
+        }
+        for (int a = 0; a < A; ++a) {
+            tc::mbar_init(tfull_bar(a), 1);
+            tc::mbar_init(tempty_bar(a), 4);
+        }
+        tc::mbar_init(mma_done_bar, 1);
+        tc::fence_mbar_init();
+    }
+    if (warp == kDecMmaWarp) {
+        tc::tmem_alloc(sbase + Lay::kTmemSlot, kTmemCols);
+        tc::tmem_relinquish();
+    }
+    if (warp >= kDecProducer0 && warp < kDecMmaWarp && lane == 0) tc::tma_prefetch_desc(&tmap_k);
+    __syncthreads();
+    block_inclusive_scan(prefix + 1, B, reinterpret_cast<int *>(smem));  // scratch: stage 0, not yet in use
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int total = prefix[B];
+    const int i0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
+    const int i1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
+    const int nsteps = i1 - i0;
+
+    if (warp >= kDecProducer0 && warp < kDecMmaWarp) {
+        // ------------------------------------------------------------ producers
+        const int pw = warp - kDecProducer0;
+        bool ok = true;
+        int carry = 0;     // sequence starts in earlier batches
+        int n_issued = 0;  // steps this warp has arrived on
+        for (int base = 0; base < nsteps && ok; base += 32) {
+            int my_b = 0, my_st = 0, my_n = 0, my_np = 0;
+            int my_pg[SP];  // every page of the step: the first warp records their validity
+#pragma unroll
+            for (int k = 0; k < SP; ++k) my_pg[k] = 0;
+            const bool valid = base + lane < nsteps;
+            if (valid) {
+                const int gi = i0 + base + lane;
+                int lo = 0, hi = B;  // prefix[lo] <= gi < prefix[hi]
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (prefix[mid] <= gi) lo = mid;
+                    else hi = mid;
+                }
+                my_b = lo;
+                my_st = gi - prefix[lo];
+                my_n = seq_len_of(lo);
+                const int pages = (my_n + kDecPage - 1) / kDecPage;
+                my_np = min(SP, pages - SP * my_st);
+                const int32_t *bt = block_table + (size_t)lo * max_pages + SP * my_st;
+#pragma unroll
+                for (int k = 0; k < SP; ++k)
+                    if (k < my_np) my_pg[k] = __ldg(bt + k);
+            }
+            // steps that begin a sequence (or the range) take the next query slot
+            const unsigned starts = __ballot_sync(0xFFFFFFFFu, valid && (my_st == 0 || base + lane == 0));
+            const int cnt = min(32, nsteps - base);
+            for (int j = 0; j < cnt; ++j) {
+                const int b = __shfl_sync(0xFFFFFFFFu, my_b, j);
+                const int st = __shfl_sync(0xFFFFFFFFu, my_st, j);
+                const int n = __shfl_sync(0xFFFFFFFFu, my_n, j);
+                const int np = __shfl_sync(0xFFFFFFFFu, my_np, j);
+                int flags = 0;  // bit i: page i of the step maps a cache page
+                int pg[PPW];
+#pragma unroll
+                for (int k = 0; k < SP; ++k) {
+                    const int p = __shfl_sync(0xFFFFFFFFu, my_pg[k], j);
+                    if (k < np && p >= 0 && p < num_pages) flags |= 1 << k;
+                    if (k / PPW == pw) pg[k % PPW] = p;
+                }
+                if (pw == 0 && ((starts >> j) & 1u)) {
+                    // the sequence's query rows, zero-padded to N, swizzled like a TMA box;
+                    // one warp copies them all, in order, so that a slot's empty
+                    // barrier is never two phases behind the wait for it
+                    const int qc = carry + __popc(starts & (0xFFFFFFFFu >> (31 - j))) - 1;
+                    const int qs = qc & 1;
+                    int got = 1;
+                    if (lane == 0)
+                        got = tc::mbar_wait_sleep(qempty_bar(qs), ((qc >> 1) & 1) ^ 1, kWaitLimitNs, kIssuerSleepNs);
+                    if (!__shfl_sync(0xFFFFFFFFu, got, 0)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t qaddr = sbase + Lay::kQ + qs * Lay::kQBytes;
+                    for (int c = lane; c < N * CPR; c += 32) {
+                        const int row = c / CPR, ch = c % CPR;
+                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                        if (row < HI) v = __ldg(reinterpret_cast<const uint4 *>(q8 + ((size_t)b * HI + row) * DI) + ch);
+                        const int sw = ch ^ ((row * DI >> 7) & (CPR - 1));
+                        st_shared_v4(qaddr + row * DI + sw * 16, v);
+                    }
+                    tc::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(qfull_bar(qs));
+                }
+                const int li = base + j, s = li % S;
+                int got = 1;
+                if (lane == 0) {
+                    // every producer waits for every step in order, so no wait
+                    // here runs two phases ahead of its barrier
+                    got = tc::mbar_wait_sleep(empty_bar(s), ((li / S) & 1) ^ 1, kWaitLimitNs, kIssuerSleepNs);
+                    if (got) {
+                        const uint32_t st_addr = sbase + s * Lay::kStageBytes;
+                        const int mine = max(0, min(PPW, np - PPW * pw));
+                        if (pw == 0)
+                            *reinterpret_cast<int4 *>(smem + s * Lay::kStageBytes + Lay::kMeta) =
+                                make_int4(b, st, n, flags);
+                        if (mine > 0) tc::mbar_arrive_expect_tx(full_bar(s), (uint32_t)mine * kPageTx);
+                        else tc::mbar_arrive(full_bar(s));
+#pragma unroll
+                        for (int k = 0; k < PPW; ++k) {
+                            const int pi = PPW * pw + k;
+                            if (pi < np) {
+                                const int p = (flags >> pi) & 1 ? pg[k] : 0;
+                                tc::tma_load_2d(st_addr + pi * kDecPage * DI, &tmap_k, 0, p * kDecPage, full_bar(s));
+                                tc::bulk_load(st_addr + Lay::kScales + pi * kDecPage * 4, skc + (size_t)p * kDecPage,
+                                              kDecPage * 4, full_bar(s));
+                            }
+                        }
+                    }
+                }
+                if (!__shfl_sync(0xFFFFFFFFu, got, 0)) {
+                    ok = false;
+                    break;
+                }
+                ++n_issued;
+            }
+            carry += __popc(starts);
+        }
+        if (lane == 0) {
+            if (!ok) record_timeout();
+            // this warp's copies have landed before the CTA may exit: only the
+            // last S steps can still be in flight, each the latest use of its stage
+            const uint64_t lim = ok ? kWaitLimitNs : 100000000ull;
+            for (int li = max(0, n_issued - S); li < n_issued; ++li)
+                (void)tc::mbar_wait(full_bar(li % S), (uint32_t)((li / S) & 1), lim);
+        }
+        __syncwarp();
+    } else if (warp == kDecMmaWarp) {
+        // ------------------------------------------------------------ UMMA
+        if (lane == 0) {
+            bool ok = true;
+            int cur_b = -1, qc = -1;
+            for (int li = 0; li < nsteps; ++li) {
+                const int s = li % S, a = li % A;
+                if (!tc::mbar_wait_sleep(full_bar(s), (li / S) & 1, kWaitLimitNs, kIssuerSleepNs)) {
+                    ok = false;
+                    break;
+                }
+                const volatile int *mp = reinterpret_cast<volatile int *>(smem + s * Lay::kStageBytes + Lay::kMeta);
+                const int4 meta = make_int4(mp[0], mp[1], mp[2], mp[3]);
+                if (meta.x != cur_b) {
+                    if (qc >= 0) tc::umma_commit(qempty_bar(qc & 1));
+                    cur_b = meta.x;
+                    ++qc;
+                    if (!tc::mbar_wait_sleep(qfull_bar(qc & 1), (qc >> 1) & 1, kWaitLimitNs, kIssuerSleepNs)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (!tc::mbar_wait_sleep(tempty_bar(a), ((li / A) & 1) ^ 1, kWaitLimitNs, kIssuerSleepNs)) {
+                    ok = false;
+                    break;
+                }
+                tc::tc_fence_after();
+                const uint32_t kaddr = sbase + s * Lay::kStageBytes;
+                const uint32_t qaddr = sbase + Lay::kQ + (qc & 1) * Lay::kQBytes;
+                const int pages = min(SP, (meta.z + kDecPage - 1) / kDecPage - SP * meta.y);
+#pragma unroll
+                for (int t = 0; t < T; ++t) {
+                    if (2 * t >= pages) break;
+                    const uint32_t d = tmem_base + (uint32_t)(a * Lay::kAccCols + t * N);
+#pragma unroll
+                    for (int ks = 0; ks < KSTEPS; ++ks)
+                        tc::umma_f8(d, tc::smem_desc_kmajor(kaddr + t * 2 * kDecPage * DI + ks * 32, DI),
+                                    tc::smem_desc_kmajor(qaddr + ks * 32, DI), IDESC, ks > 0 ? 1u : 0u);
+                }
+                tc::umma_commit(empty_bar(s));
+                tc::umma_commit(tfull_bar(a));
+            }
+            if (!ok) record_timeout();
+            tc::umma_commit(mma_done_bar);
+            (void)tc::mbar_wait(mma_done_bar, 0, kWaitLimitNs);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int grp = warp / 4;
+        const int qw = warp & 3;  // TMEM lane quarter
+        const uint32_t lane_base = tmem_base + ((uint32_t)(qw * 32) << 16);
+        int cur_b = -1;
+        float wv[N];
+        float sqb = 0.f;
+#pragma unroll
+        for (int h = 0; h < N; ++h) wv[h] = 0.f;
+        bool ok = true;
+        for (int li = grp; li < nsteps; li += G) {
+            const int s = li % S, a = li % A;
+            if (!tc::mbar_wait(tfull_bar(a), (li / A) & 1, kWaitLimitNs) ||
+                !tc::mbar_wait(full_bar(s), (li / S) & 1, kWaitLimitNs)) {
+                ok = false;
+                break;
+            }
+            tc::tc_fence_after();
+            const uint8_t *stp = smem + s * Lay::kStageBytes;
+            const int4 meta = *reinterpret_cast<const int4 *>(stp + Lay::kMeta);
+            float sk[T];
+#pragma unroll
+            for (int t = 0; t < T; ++t) sk[t] = reinterpret_cast<const float *>(stp + Lay::kScales)[t * 128 + qw * 32 + lane];
+            const int step_pages = min(SP, (meta.z + kDecPage - 1) / kDecPage - SP * meta.y);
+            float v[T];
+#pragma unroll
+            for (int t = 0; t < T; ++t) {
+                float part[4] = {0.f, 0.f, 0.f, 0.f};
+                if (2 * t < step_pages) {
+#pragma unroll
+                    for (int c0 = 0; c0 < N; c0 += 16) {
+                        float acc[16];
+                        tc::tmem_ld16(lane_base + (uint32_t)(a * Lay::kAccCols + t * N + c0), acc);
+                        tc::tmem_wait_ld();
+                        if (meta.x != cur_b) {
+                            cur_b = meta.x;
+#pragma unroll
+                            for (int h = 0; h < N; ++h) wv[h] = h < HI ? __ldg(w + (size_t)cur_b * HI + h) : 0.f;
+                            sqb = __ldg(sq + cur_b);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) part[j & 3] = fmaf(wv[c0 + j], fmaxf(acc[j], 0.f), part[j & 3]);
+                    }
+                }
+                v[t] = (part[0] + part[1]) + (part[2] + part[3]);
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(tempty_bar(a));
+                tc::mbar_arrive(empty_bar(s));
+            }
+#pragma unroll
+            for (int t = 0; t < T; ++t) {
+                const int pi = 2 * t + (qw >> 1);  // page of the step
+                const int tok = (SP * meta.y + pi) * kDecPage + (qw & 1) * 32 + lane;
+                if (tok < meta.z)
+                    scores[(size_t)cur_b * ld + tok] = ((meta.w >> pi) & 1) ? v[t] * sqb * sk[t] : -INFINITY;
+            }
+        }
+        if (!ok) record_timeout();
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == kDecMmaWarp) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (fn == nullptr) {
@@ -404,6 +811,21 @@ cudaError_t launch_tc(const uint8_t *q8, const float *sq, const float *w, const 
     return cudaGetLastError();
 }
 
+template <int N, int DI>
+cudaError_t launch_decode_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8c, const float *skc,
+                             const int32_t *block_table, int max_pages, int num_pages, const int32_t *seq_lens,
+                             int max_seq_len, int B, int HI, float *scores, int64_t ld, cudaStream_t stream) {
+    CUtensorMap mk;
+    if (!make_map(&mk, k8c, (uint64_t)num_pages * kDecPage, DI, kDecPage)) return cudaErrorInvalidValue;
+    constexpr int smem = DecLayout<N, DI>::kAlloc > 116 * 1024 ? DecLayout<N, DI>::kAlloc : 116 * 1024;
+    cudaError_t e =
+        cudaFuncSetAttribute(indexer_decode_tc_kernel<N, DI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    indexer_decode_tc_kernel<N, DI><<<sm_count(), kDecThreads, smem, stream>>>(
+        mk, q8, sq, w, skc, block_table, max_pages, num_pages, seq_lens, max_seq_len, B, HI, scores, ld);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 bool indexer_tc_supported(int HI, int dI) {
@@ -437,6 +859,38 @@ cudaError_t indexer_tc_take_error(unsigned int *flag) {
     cudaError_t e = cudaMemcpyFromSymbol(flag, g_indexer_tc_error, sizeof(unsigned int));
     if (e != cudaSuccess) return e;
     return cudaMemcpyToSymbol(g_indexer_tc_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace dsa
+
+namespace dsa {
+
+bool indexer_decode_tc_supported(int HI, int dI, int B, int max_seq_len) {
+    const bool shape = (HI == 4 || HI == 8 || HI == 16 || HI == 32 || HI == 64) && (dI == 32 || dI == 64 || dI == 128);
+    // the step prefix lives in shared memory and is counted in int
+    return shape && B <= kDecMaxB && (int64_t)B * ((max_seq_len + kDecPage - 1) / kDecPage) < (1ll << 31);
+}
+
+cudaError_t launch_indexer_decode_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8c,
+                                     const float *skc, const int32_t *block_table, int max_pages, int num_pages,
+                                     const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI, float *scores,
+                                     int64_t ld, cudaStream_t stream) {
+    if (B == 0 || max_seq_len == 0) return cudaSuccess;
+    auto by_di = [&](auto n) -> cudaError_t {
+        constexpr int NN = decltype(n)::value;
+        switch (dI) {
+            case 32: return launch_decode_tc<NN, 32>(q8, sq, w, k8c, skc, block_table, max_pages, num_pages, seq_lens,
+                                                     max_seq_len, B, HI, scores, ld, stream);
+            case 64: return launch_decode_tc<NN, 64>(q8, sq, w, k8c, skc, block_table, max_pages, num_pages, seq_lens,
+                                                     max_seq_len, B, HI, scores, ld, stream);
+            case 128: return launch_decode_tc<NN, 128>(q8, sq, w, k8c, skc, block_table, max_pages, num_pages,
+                                                       seq_lens, max_seq_len, B, HI, scores, ld, stream);
+            default: return cudaErrorInvalidValue;
+        }
+    };
+    if (HI <= 16) return by_di(std::integral_constant<int, 16>{});
+    if (HI == 32) return by_di(std::integral_constant<int, 32>{});
+    return by_di(std::integral_constant<int, 64>{});
 }
 
 }  // namespace dsa

@@ -25,6 +25,11 @@ cudaError_t launch_indexer_prefill_tc(const uint8_t *q8, const float *sq, const 
                                       const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
                                       float *scores, int64_t ld, float *row_stats, cudaStream_t stream);
 cudaError_t indexer_tc_take_error(unsigned int *flag);
+bool indexer_decode_tc_supported(int HI, int dI, int B, int max_seq_len);
+cudaError_t launch_indexer_decode_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8c,
+                                     const float *skc, const int32_t *block_table, int max_pages, int num_pages,
+                                     const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI, float *scores,
+                                     int64_t ld, cudaStream_t stream);
 
 // topk.cu
 size_t topk_workspace_bytes(int n_rows, int max_len, int k);

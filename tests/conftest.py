@@ -34,3 +34,14 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(autouse=True)
+def _no_expired_device_waits(request):
+    """After every GPU test: no kernel of the library gave up a bounded wait
+    (such a kernel stops early and sets a device flag, read and cleared here)."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    from sparse_long_context_03_b200 import dsa
+    dsa.check_device_error()

@@ -346,6 +346,75 @@ def test_decode_small_matches_oracle(cfg_id, lens, k):
     check_attention(o3.float().cpu().numpy(), Oref2, l3.cpu().numpy(), lref2, "decode attention stage")
 
 
+def _paged_exact(HI, dI, lens, seed, unmapped=()):
+    """Exact-arithmetic keys (see inputs.exact_indexer_inputs) dealt to cache
+    pages in a random order and shared by every sequence; sequence b's query
+    is the exact query row of position lens[b] - 1.  `unmapped` lists
+    (sequence, logical page, page id) entries written into the block table."""
+    L = max(lens)
+    P = (L + 63) // 64
+    d = {k: v.numpy() for k, v in inputs.exact_indexer_inputs(L, HI, dI, seed=seed).items()}
+    rng = np.random.default_rng(seed)
+    n_pages = P + 2
+    perm = rng.permutation(n_pages).astype(np.int32)
+    k8c = np.zeros((n_pages, 64, dI), np.uint8)
+    skc = np.ones((n_pages, 64), np.float32)
+    for j in range(P):
+        lo, hi = j * 64, min(L, j * 64 + 64)
+        k8c[perm[j], : hi - lo] = d["k8"][lo:hi]
+        skc[perm[j], : hi - lo] = d["sk"][lo:hi]
+    B = len(lens)
+    bt = np.tile(perm[:P], (B, 1)).astype(np.int32)
+    for b, j, v in unmapped:
+        bt[b, j] = v
+    t = np.array(lens) - 1
+    return dict(q8=d["q8"][t].copy(), sq=d["sq"][t].copy(), w=d["w"][t].copy(), k8_cache=k8c, sk_cache=skc,
+                block_table=bt, seq_lens=np.array(lens, np.int32), max_seq_len=L, num_pages=n_pages)
+
+
+def _decode_scores_gpu(h):
+    g = {k: (torch.from_numpy(v).to(DEV) if isinstance(v, np.ndarray) else v) for k, v in h.items()}
+    B = len(h["seq_lens"])
+    ld = (h["max_seq_len"] + 3) // 4 * 4
+    sc = torch.full((B, ld), float("nan"), dtype=torch.float32, device=DEV)
+    dsa.decode_indexer_scores(g["q8"], g["sq"], g["w"], g["k8_cache"], g["sk_cache"], g["block_table"],
+                              g["seq_lens"], h["max_seq_len"], sc)
+    torch.cuda.synchronize()
+    return sc.cpu().numpy()
+
+
+@pytest.mark.parametrize("HI,dI", [(4, 32), (8, 64), (16, 128), (32, 64), (64, 128), (32, 32), (64, 64)])
+def test_decode_indexer_exact_inputs_bit_exact(HI, dI):
+    # lengths around page and 128-key item boundaries, one long sequence;
+    # unmapped entries: past the cache, negative, and a whole odd last page
+    lens = [1, 63, 64, 65, 127, 128, 129, 700, 1000, 257]
+    P = (max(lens) + 63) // 64
+    n_pages = P + 2
+    unmapped = [(7, 3, n_pages), (8, 10, -3), (8, 0, n_pages + 100), (9, 4, -1), (2, 1, 2 ** 31 - 1)]
+    h = _paged_exact(HI, dI, lens, seed=300 + HI + dI, unmapped=unmapped)
+    ref = oracle.decode_indexer(h["q8"], h["sq"], h["w"], h["k8_cache"], h["sk_cache"], h["block_table"],
+                                h["seq_lens"])
+    got = _decode_scores_gpu(h)
+    for b, n in enumerate(lens):
+        assert np.array_equal(got[b, :n], ref[b, :n]), f"sequence {b}"
+    assert np.isneginf(ref[7, 3 * 64]) and np.isneginf(ref[8, 0]) and np.isneginf(ref[9, 256])
+
+
+@pytest.mark.parametrize("B", [4096, 4100])
+def test_decode_indexer_large_batches(B):
+    # 4096 sequences is the tensor-core path's largest batch; 4100 takes the
+    # other path.  Both must give the same scores.
+    cfg = inputs.config(0)
+    lens = np.random.default_rng(B).integers(1, 300, B).tolist()
+    d = inputs.decode_inputs(cfg, seq_lens=lens, seed=B)
+    h = {k: (H(v) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    ref = oracle.decode_indexer(h["q8"], h["sq"], h["w"], h["k8_cache"], h["sk_cache"], h["block_table"],
+                                h["seq_lens"])
+    got = _decode_scores_gpu(h)
+    for b, n in enumerate(lens):
+        check_scores(got[b, :n], ref[b, :n], f"sequence {b}")
+
+
 # ----------------------------------------------------------------------------
 # full-size workloads, sampled rows, benchmark launch configuration
 # ----------------------------------------------------------------------------

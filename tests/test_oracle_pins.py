@@ -363,6 +363,37 @@ def test_decode_paged_equals_contiguous(oracle_mod):
         np.testing.assert_array_equal(ld_, lc)
 
 
+def test_decode_unmapped_pages_have_no_keys(oracle_mod):
+    # Library convention, not from the pages: a block-table entry outside the
+    # cache's pages maps no key.  Its tokens score -inf, the others keep the
+    # scores of the fully mapped table, and attention over an index set that
+    # names them equals contiguous attention over the set without them.
+    cfg = inputs.config(0)
+    d = inputs.decode_inputs(cfg, seq_lens=[200], seed=6)
+    n = {k: (_np(v) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    full = oracle_mod.decode_indexer(n["q8"], n["sq"], n["w"], n["k8_cache"], n["sk_cache"],
+                                     n["block_table"], n["seq_lens"])
+    bt = n["block_table"].copy()
+    P = n["k8_cache"].shape[0]
+    bt[0, 1] = P       # tokens 64..127
+    bt[0, 3] = -5      # tokens 192..199
+    I = oracle_mod.decode_indexer(n["q8"], n["sq"], n["w"], n["k8_cache"], n["sk_cache"], bt, n["seq_lens"])
+    gone = np.zeros(200, bool)
+    gone[64:128] = True
+    gone[192:200] = True
+    assert np.all(np.isneginf(I[0, gone]))
+    np.testing.assert_array_equal(I[0, ~gone], full[0, ~gone])
+    idx = np.array([[3, 70, 130, 195, 199, 10, 127, 64]], np.int32)
+    Od, lse_d = oracle_mod.decode_attention(n["q"], n["k_cache"], n["v_cache"], bt, n["seq_lens"], idx,
+                                            cfg.sm_scale)
+    keep = np.array([[3, 130, 10, -1, -1, -1, -1, -1]], np.int32)
+    Kc = _contiguous_from_pages(n["k_cache"], n["block_table"][0], 200)
+    Vc = _contiguous_from_pages(n["v_cache"], n["block_table"][0], 200)
+    Oc, lc = oracle_mod.sparse_attention(n["q"], Kc, Vc, keep, 199, cfg.sm_scale)
+    np.testing.assert_array_equal(Od, Oc)
+    np.testing.assert_array_equal(lse_d, lc)
+
+
 def test_oracle_results_do_not_depend_on_thread_count(oracle_mod):
     cfg = inputs.config(0)
     d = inputs.prefill_inputs(cfg, L=96, seed=31)
