@@ -264,11 +264,11 @@ def run_prefill_e2e(pb, steps, warmup):
 
 
 class DecodeBench:
-    def __init__(self, cfg, seed, device):
+    def __init__(self, cfg, seed, device, batch=None):
         from sparse_long_context_03_b200 import dsa, inputs
         self.dsa = dsa
         self.cfg = cfg
-        self.d = inputs.decode_inputs(cfg, device=device, seed=seed)
+        self.d = inputs.decode_inputs(cfg, device=device, seed=seed, B=batch)
         B = self.d["q"].shape[0]
         self.B = B
         self.ws = torch.empty(dsa.decode_workspace_size(B, self.d["max_seq_len"], cfg.Hq, cfg.Hkv, cfg.D, cfg.k),
@@ -429,6 +429,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--chunk-rows", type=int, default=None,
                     help="query rows per indexer/top-k chunk (default: a 4 GiB score block)")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="sequences in the decode workload (default: the decode-b32 layer's 32)")
     args = ap.parse_args()
 
     if args.impl == "reference":
@@ -468,7 +470,7 @@ def main():
         del pb
         torch.cuda.empty_cache()
         dcfg = inputs.config(3)
-        db = DecodeBench(dcfg, seed=rank_seed(dcfg, rank), device="cuda")
+        db = DecodeBench(dcfg, seed=rank_seed(dcfg, rank), device="cuda", batch=args.decode_batch)
         us = 1e3 * max_over_ranks(run_decode_timed(db, max(args.steps, 20), max(args.warmup, 3)), world)
         byts = db.algorithmic_bytes()
         decode = {"workload": f"{dcfg.name}: B={db.B}, cached lengths U[{dcfg.len_lo},{dcfg.len_hi}] "
