@@ -205,6 +205,33 @@ class PrefillBench:
         return gather + qo + 4 * c.k * n              # + index rows
 
 
+TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "dram_traffic.txt")
+STAGE_KERNEL = {"attention": ("sparse_prefill_kernel", "attention.cu"),
+                "indexer": ("indexer_tc_kernel", "indexer_tc.cu"),
+                "topk": ("topk_rows_kernel", "topk.cu")}
+
+
+def measured_traffic(stage, workload):
+    """DRAM bytes (read + write) per launch of a stage's kernel on this
+    workload, from the ncu capture recorded in profiles/dram_traffic.txt --
+    only if that capture was taken on the kernel's current source (its
+    sha256 is recorded beside the figure); None otherwise."""
+    import hashlib
+    kernel, src = STAGE_KERNEL[stage]
+    try:
+        from sparse_long_context_03_b200 import build
+        digest = hashlib.sha256(open(os.path.join(build.CSRC, src), "rb").read()).hexdigest()
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 5 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload \
+                        and parts[4] == digest:
+                    return int(parts[2]) + int(parts[3])
+    except OSError:
+        return None
+    return None
+
+
 def run_prefill_timed(pb, steps, warmup, world, gpu_index):
     for _ in range(warmup):
         pb.step()
@@ -455,7 +482,12 @@ def main():
     dominant = max(stages, key=lambda k: stages[k]["ms_total"])
     dom = dict(stages[dominant])
     dom_line = {"kernel": dominant, "bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"],
-                "unit": dom["unit"], "frac": dom["frac"], "traffic": None, "peak_source": dom["peak_note"]}
+                "unit": dom["unit"], "frac": dom["frac"], "traffic": measured_traffic(dominant, cfg.name),
+                "peak_source": dom["peak_note"]}
+    if dominant == "attention":
+        dom_line["note"] = ("achieved = algorithmic gather bytes (every selected K/V row once per query and KV "
+                            "group) / time; most rows are served from L2, so it can exceed the HBM copy peak; "
+                            "traffic = DRAM bytes per launch from ncu")
 
     e2e = None
     if not args.no_e2e:

@@ -226,12 +226,15 @@ template <int D>
 __global__ void __launch_bounds__(kWarpsPerCta * 32) sparse_prefill_kernel(
     const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K, const uint16_t *__restrict__ V,
     const int32_t *__restrict__ idx, int row_begin, int n_rows, int Hq, int Hkv, int k, float scale_log2,
-    uint16_t *__restrict__ O, float *__restrict__ lse) {
+    uint16_t *__restrict__ O, float *__restrict__ lse, int group_major) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = lane_id();
     const int pair = blockIdx.x * kWarpsPerCta + warp;
     if (pair >= n_rows * Hkv) return;
-    const int r = pair / Hkv, g = pair % Hkv;
+    // group-major: the warps resident at one time share one KV group, whose
+    // K and V rows then fit in L2 even when the whole K and V do not
+    const int r = group_major ? pair % n_rows : pair / Hkv;
+    const int g = group_major ? pair / n_rows : pair % Hkv;
     const int t = row_begin + r;
     const int G = Hq / Hkv;
     uint8_t *wsmem = smem + warp * warp_smem_bytes<D>();
@@ -390,6 +393,10 @@ cudaError_t launch_sparse_prefill(const uint16_t *Q, const uint16_t *K, const ui
     if (n_rows == 0) return cudaSuccess;
     const int64_t pairs = (int64_t)n_rows * Hkv;
     const int grid = (int)((pairs + kWarpsPerCta - 1) / kWarpsPerCta);
+    // Walk the pairs group by group once the visible K and V rows outgrow
+    // half of L2 (at 128K tokens they are 268 MB; one group's share fits).
+    const int64_t kv_bytes = 2ll * (row_begin + n_rows) * Hkv * D * 2;
+    const bool group_major = Hkv > 1 && kv_bytes > (64ll << 20);
     cudaError_t err = cudaSuccess;
     const bool ok = dispatch_d(D, [&](auto dc) {
         constexpr int DD = decltype(dc)::value;
@@ -397,7 +404,8 @@ cudaError_t launch_sparse_prefill(const uint16_t *Q, const uint16_t *K, const ui
         err = cudaFuncSetAttribute(sparse_prefill_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err != cudaSuccess) return true;
         sparse_prefill_kernel<DD><<<grid, kWarpsPerCta * 32, smem, stream>>>(Q, K, V, idx, row_begin, n_rows, Hq,
-                                                                             Hkv, k, sm_scale * kLog2e, O, lse);
+                                                                             Hkv, k, sm_scale * kLog2e, O, lse,
+                                                                             group_major ? 1 : 0);
         err = cudaGetLastError();
         return true;
     });

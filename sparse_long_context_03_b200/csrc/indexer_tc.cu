@@ -56,16 +56,21 @@ constexpr uint32_t kTmemCols = 512;
 // tiles (one 256-row TMA box, 2 x dI/32 MMAs into an accumulator pair, one
 // commit) halves that cost per MMA.
 
-// Columns per epilogue warp and the warp counts for HI heads per query.  With
-// 18 warps, two of the four schedulers hold five warps, whose 16K-register
-// files cap a thread at 96 registers (HI <= 32); HI = 64 has 10 warps.
+// Columns per epilogue warp and the warp counts for HI heads per query.  Two
+// MMA warps take alternate steps, each into its own accumulator pair: the
+// fixed cost of one issuing thread per step (two mbarrier waits, fences, two
+// commits: about 900 cycles) is what paced a single MMA warp, and two of them
+// overlap it.  With 19 warps, three of the four schedulers hold five warps,
+// whose 16K-register files cap a thread at 96 registers (HI <= 32); HI = 64
+// has 11 warps.
 template <int HI>
 struct EpiShape {
     static constexpr int CW = HI > 32 ? HI : 32;
     static constexpr int kEpiWarps = 4 * (kTileN / CW);
-    static constexpr int kThreads = (kEpiWarps + 2) * 32;
+    static constexpr int kThreads = (kEpiWarps + 3) * 32;
     static constexpr int kProducerWarp = kEpiWarps;
-    static constexpr int kMmaWarp = kEpiWarps + 1;
+    static constexpr int kMmaWarp = kEpiWarps + 1;  // and kMmaWarp + 1
+    static constexpr int kMaxRegs = kThreads > 512 ? 96 : 168;
 };
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 constexpr uint32_t kIssuerSleepNs = 32;            // back-off of the TMA and MMA warps
@@ -74,9 +79,11 @@ constexpr uint32_t kIssuerSleepNs = 32;            // back-off of the TMA and MM
 template <int DI>
 struct Layout {
     static constexpr int kTileBytes = kStepKeys * DI;  // one step of keys
-    static constexpr int kStages = (200 * 1024 - 2 * kTileN * DI) / kTileBytes > 8
-                                       ? 8
-                                       : (200 * 1024 - 2 * kTileN * DI) / kTileBytes;
+    // even: stage s then serves steps of one parity only, i.e. of one MMA
+    // warp, which waits for its phases in order
+    static constexpr int kStages = ((200 * 1024 - 2 * kTileN * DI) / kTileBytes > 8
+                                        ? 8
+                                        : (200 * 1024 - 2 * kTileN * DI) / kTileBytes) & ~1;
     static constexpr int kQBytes = kTileN * DI;
     static constexpr int kKeys = 0;
     static constexpr int kQ = kKeys + kStages * kTileBytes;
@@ -90,7 +97,7 @@ struct Layout {
 __device__ __forceinline__ void record_timeout() { atomicOr(&g_indexer_tc_error, 1u); }
 
 template <int HI, int DI>
-__global__ void __launch_bounds__(EpiShape<HI>::kThreads, 1) indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
+__global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                                                  const __grid_constant__ CUtensorMap tmap_q,
                                                                  const float *__restrict__ sq,
                                                                  const float *__restrict__ w,
@@ -131,13 +138,13 @@ __global__ void __launch_bounds__(EpiShape<HI>::kThreads, 1) indexer_tc_kernel(c
         }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(qfull_bar(b), 1);
-            tc::mbar_init(qempty_bar(b), 1);
+            tc::mbar_init(qempty_bar(b), 2);  // one commit per MMA warp
         }
         for (int b = 0; b < kPairs; ++b) {
             tc::mbar_init(tfull_bar(b), 1);
             tc::mbar_init(tempty_bar(b), kEpiWarps);
         }
-        tc::mbar_init(mma_done_bar, 1);
+        tc::mbar_init(mma_done_bar, 2);
         tc::fence_mbar_init();
     }
     if (warp == kMmaWarp) {
@@ -194,11 +201,14 @@ __global__ void __launch_bounds__(EpiShape<HI>::kThreads, 1) indexer_tc_kernel(c
             for (int j = max(0, q_issued - 2); j < q_issued; ++j)
                 (void)tc::mbar_wait(qfull_bar(j & 1), (uint32_t)((j >> 1) & 1), lim);
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
         // ------------------------------------------------------------ UMMA
+        // MMA warp mw issues the steps it with it % 2 == mw, into pair mw.
+        // Both warps walk every query block and wait for its query tile, so
+        // each waits for every barrier phase it uses in order.
+        static_assert(kPairs == 2, "one accumulator pair per MMA warp");
+        const int mw = warp - kMmaWarp;
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
             int it = 0, bi = 0;
             bool ok = true;
             for (int i = blockIdx.x; i < nb && ok; i += gridDim.x, ++bi) {
@@ -214,10 +224,12 @@ __global__ void __launch_bounds__(EpiShape<HI>::kThreads, 1) indexer_tc_kernel(c
                 tc::tc_fence_after();
                 const uint32_t qaddr = sbase + Lay::kQ + qs * Lay::kQBytes;
                 for (int st = 0; st < nstep; ++st, ++it) {
-                    const int pr = it % kPairs;
+                    if ((it & 1) != mw) continue;
+                    const int pr = mw;
+                    const int stage = it % kStages;
                     if (!tc::mbar_wait_sleep(tempty_bar(pr), ((it / kPairs) & 1) ^ 1, kWaitLimitNs,
                                              kIssuerSleepNs) ||
-                        !tc::mbar_wait_sleep(full_bar(stage), phase, kWaitLimitNs, kIssuerSleepNs)) {
+                        !tc::mbar_wait_sleep(full_bar(stage), (it / kStages) & 1, kWaitLimitNs, kIssuerSleepNs)) {
                         ok = false;
                         break;
                     }
@@ -235,7 +247,6 @@ __global__ void __launch_bounds__(EpiShape<HI>::kThreads, 1) indexer_tc_kernel(c
                     }
                     tc::umma_commit(empty_bar(stage));
                     tc::umma_commit(tfull_bar(pr));
-                    if (++stage == kStages) { stage = 0; phase ^= 1; }
                 }
                 tc::umma_commit(qempty_bar(qs));
             }
