@@ -296,25 +296,19 @@ __device__ void finish_row(TopkSmem &sm, const int32_t *alist, uint32_t cnt, uin
     }
 }
 
-__global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__restrict__ scores, int64_t ld,
-                                                            int row_begin, const int32_t *__restrict__ row_len,
-                                                            int max_len, int k, int32_t *__restrict__ idx,
-                                                            const float *__restrict__ row_stats) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
-    int32_t *alist = reinterpret_cast<int32_t *>(smem_raw + sizeof(TopkSmem));
+// Threshold bucket of one row (n > k): the value range (from the indexer's
+// row statistics when given), then a histogram over kNB linear buckets of it
+// and the bucket Bt holding the k-th largest entry.  Returns false when the
+// row was finished here (every entry equal, or the exact whole-row path).
+struct RowThreshold {
+    float vmin, scale;
+    uint32_t Bt, need, n_above, cnt;
+};
 
-    const int r = blockIdx.x;
-    const int n = row_length(row_len, r, row_begin, max_len);
-    const float *row = scores + (size_t)r * ld;
-    int32_t *out = idx + (size_t)r * k;
+__device__ bool row_threshold(const float *row, int n, int k, int r, const float *row_stats, TopkSmem &sm,
+                              int32_t *out, RowThreshold &t) {
     const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
-
-    if (n <= k) {  // short row: everything visible is selected
-        for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
-        return;
-    }
-
+    float scale;
     // ---- pass 1: value range (from the indexer's row statistics when given)
     float vmin = INFINITY, vmax = -INFINITY;
     if (row_stats != nullptr) {
@@ -356,15 +350,15 @@ __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__rest
     __syncthreads();
     if (vmin == vmax) {  // every entry ties: the k lowest indices
         for (int i = tid; i < k; i += kThreads) out[i] = i;
-        return;
+        return false;
     }
     const float range = vmax - vmin;
     if (!(range < INFINITY)) {  // span overflows fp32: exact slow path
         topk_row_radix(row, n, k, out, sm);
-        return;
+        return false;
     }
     // slightly below kNB / range so that vmax itself maps below kNB
-    const float scale = __fdiv_rn((float)kNB * 0.99999f, range);
+    scale = __fdiv_rn((float)kNB * 0.99999f, range);
 
     // ---- pass 2: bucket histogram
     for (int i0 = tid * kVec; i0 < n; i0 += kChunk) {
@@ -376,16 +370,45 @@ __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__rest
     }
     __syncthreads();
     find_threshold_bin(sm.hist, (uint32_t)k, sm.red, sm.bcast);
-    const uint32_t Bt = sm.bcast[0];
-    const uint32_t need = sm.bcast[1];       // taken from the threshold bucket
-    const uint32_t n_above = sm.bcast[2];    // entries in buckets above it
-    const uint32_t cnt = sm.hist[Bt];
+    t.Bt = sm.bcast[0];
+    t.need = sm.bcast[1];       // taken from the threshold bucket
+    t.n_above = sm.bcast[2];    // entries in buckets above it
+    t.cnt = sm.hist[t.Bt];
     __syncthreads();
 
-    if (cnt > (uint32_t)kCap) {
+    if (t.cnt > (uint32_t)kCap) {
         topk_row_radix(row, n, k, out, sm);
+        return false;
+    }
+    t.vmin = vmin;
+    t.scale = scale;
+    return true;
+
+}
+
+__global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__restrict__ scores, int64_t ld,
+                                                            int row_begin, const int32_t *__restrict__ row_len,
+                                                            int max_len, int k, int32_t *__restrict__ idx,
+                                                            const float *__restrict__ row_stats) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    int32_t *alist = reinterpret_cast<int32_t *>(smem_raw + sizeof(TopkSmem));
+
+    const int r = blockIdx.x;
+    const int n = row_length(row_len, r, row_begin, max_len);
+    const float *row = scores + (size_t)r * ld;
+    int32_t *out = idx + (size_t)r * k;
+    const int tid = threadIdx.x;
+
+    if (n <= k) {  // short row: everything visible is selected
+        for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
         return;
     }
+
+    RowThreshold th;
+    if (!row_threshold(row, n, k, r, row_stats, sm, out, th)) return;
+    const float vmin = th.vmin, scale = th.scale;
+    const uint32_t Bt = th.Bt, need = th.need, n_above = th.n_above, cnt = th.cnt;
 
     // ---- pass 3: ordered collect
     uint32_t run_a = 0, run_c = 0;
@@ -422,6 +445,156 @@ __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__rest
     finish_row(sm, alist, cnt, need, n_above, out);
 }
 
+
+// ---------------------------------------------------------------------------
+// Many rows of moderate length (prefill chunks): the collect pass marks the
+// selected entries in a bitmap of the row instead of building ordered lists.
+//
+// After the histogram, every entry above the threshold bucket is a winner:
+// its bit is set with one atomicOr per thread and chunk (a thread's kVec = 16
+// entries lie in one 32-bit word).  Threshold-bucket entries go, in any
+// order, to the candidate list through one atomicAdd per warp.  The chosen
+// candidates -- larger key first, then lower index -- set their bits too,
+// and one scan of the bitmap writes the k indices in ascending order.  No
+// block-wide barrier runs inside the pass over the row.  Rows whose tied
+// candidates are too many to rank directly take the whole-row radix path.
+// ---------------------------------------------------------------------------
+
+constexpr int kMaxTiedRanked = 512;     // tied candidates ranked pairwise
+// Rows up to 524288 entries: the bitmap (64 KB) and the lists still fit twice
+// per SM up to 262144 entries, once beyond.
+constexpr int kBitmapSmemMax = 124 * 1024;
+
+__host__ __device__ constexpr int bitmap_words(int max_len) { return ((max_len + 31) / 32 + 3) / 4 * 4; }
+__host__ __device__ constexpr size_t bitmap_smem_bytes(int max_len) {
+    return sizeof(TopkSmem) + sizeof(uint32_t) * (size_t)bitmap_words(max_len);
+}
+
+__global__ void __launch_bounds__(kThreads) topk_rows_bitmap_kernel(const float *__restrict__ scores, int64_t ld,
+                                                                   int row_begin,
+                                                                   const int32_t *__restrict__ row_len,
+                                                                   int max_len, int k, int32_t *__restrict__ idx,
+                                                                   const float *__restrict__ row_stats) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    uint32_t *bits = reinterpret_cast<uint32_t *>(smem_raw + sizeof(TopkSmem));
+
+    const int r = blockIdx.x;
+    const int n = row_length(row_len, r, row_begin, max_len);
+    const float *row = scores + (size_t)r * ld;
+    int32_t *out = idx + (size_t)r * k;
+    const int tid = threadIdx.x, lane = lane_id();
+
+    if (n <= k) {  // short row: everything visible is selected
+        for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
+        return;
+    }
+    RowThreshold th;
+    if (!row_threshold(row, n, k, r, row_stats, sm, out, th)) return;
+    const uint32_t Bt = th.Bt, need = th.need, cnt = th.cnt;
+
+    const int words = (n + 31) / 32;
+    for (int w = tid; w < words; w += kThreads) bits[w] = 0u;
+    if (tid == 0) sm.bcast[3] = 0u;  // candidates written so far
+    __syncthreads();
+
+    // ---- collect: winners into the bitmap, candidates into the list.  The
+    // trip count is the same for every thread: the warp shuffles below need
+    // all 32 lanes in every iteration.
+    for (int base = 0; base < n; base += kChunk) {
+        const int i0 = base + tid * kVec;
+        float x[kVec] = {};
+        const int m = i0 < n ? load_vals(row, i0, n, x) : 0;
+        uint32_t win = 0u, cmask = 0u;
+#pragma unroll
+        for (int j = 0; j < kVec; ++j) {
+            const uint32_t b = bucket_of(x[j], th.vmin, th.scale);
+            if (j < m && b > Bt) win |= 1u << j;
+            if (j < m && b == Bt) cmask |= 1u << j;
+        }
+        if (win) atomicOr(&bits[i0 >> 5], win << (i0 & 31));
+        // warp-aggregated slots for the candidates
+        const uint32_t c = __popc(cmask);
+        uint32_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t wtot = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        uint32_t slot = 0u;
+        if (lane == 31 && wtot) slot = atomicAdd(&sm.bcast[3], wtot);
+        slot = __shfl_sync(0xFFFFFFFFu, slot, 31) + incl - c;
+        while (cmask) {
+            const int j = __ffs(cmask) - 1;
+            cmask &= cmask - 1u;
+            sm.ckey[slot] = order_key(x[j]);
+            sm.cidx[slot] = i0 + j;
+            ++slot;
+        }
+    }
+    __syncthreads();
+
+    // ---- choose `need` of the cnt candidates: larger key first, lower index on ties
+    if (cnt <= (uint32_t)kSmallCand) {
+        const int i = tid;
+        if (i < (int)cnt) {
+            const uint32_t ki = sm.ckey[i];
+            const int32_t xi = sm.cidx[i];
+            uint32_t rank = 0;
+            for (int j = 0; j < (int)cnt; ++j) {
+                const uint32_t kj = sm.ckey[j];
+                rank += (kj > ki) || (kj == ki && sm.cidx[j] < xi);
+            }
+            if (rank < need) atomicOr(&bits[xi >> 5], 1u << (xi & 31));
+        }
+    } else {
+        uint32_t T, quota;
+        select_in_candidates(sm, (int)cnt, need, T, quota);
+        // how many candidates tie at T
+        uint32_t tied = 0;
+        for (int i = tid; i < (int)cnt; i += kThreads) tied += sm.ckey[i] == T;
+        tied = __reduce_add_sync(0xFFFFFFFFu, tied);
+        if (lane == 0) sm.red[tid >> 5] = tied;
+        __syncthreads();
+        uint32_t n_tied = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) n_tied += sm.red[w];
+        __syncthreads();
+        if (n_tied > (uint32_t)kMaxTiedRanked) {
+            topk_row_radix(row, n, k, out, sm);
+            return;
+        }
+        for (int i = tid; i < (int)cnt; i += kThreads) {
+            const uint32_t ki = sm.ckey[i];
+            const int32_t xi = sm.cidx[i];
+            bool take = ki > T;
+            if (ki == T) {
+                uint32_t before = 0;
+                for (int j = 0; j < (int)cnt; ++j) before += sm.ckey[j] == T && sm.cidx[j] < xi;
+                take = before < quota;
+            }
+            if (take) atomicOr(&bits[xi >> 5], 1u << (xi & 31));
+        }
+    }
+    __syncthreads();
+
+    // ---- the k set bits, in index order
+    const int per = (words + kThreads - 1) / kThreads;
+    const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
+    uint32_t mine = 0;
+    for (int w = w0; w < w1; ++w) mine += __popc(bits[w]);
+    uint32_t tot;
+    uint32_t pos = block_scan_packed(mine, sm.red, &tot);
+    for (int w = w0; w < w1; ++w) {
+        uint32_t v = bits[w];
+        while (v) {
+            const int b = __ffs(v) - 1;
+            v &= v - 1u;
+            out[pos++] = w * 32 + b;
+        }
+    }
+}
 
 // ---------------------------------------------------------------------------
 // Long rows, few of them (decode): one thread-block cluster per row.
@@ -642,6 +815,15 @@ cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_ro
         if (e != cudaSuccess) return e;
         topk_rows_cluster_kernel<<<n_rows * kClusterSize, kThreads, csmem, stream>>>(scores, ld, row_begin, row_len,
                                                                                        max_len, k, idx, row_stats);
+        return cudaGetLastError();
+    }
+    if (bitmap_smem_bytes(max_len) <= (size_t)kBitmapSmemMax) {
+        const size_t bsmem = bitmap_smem_bytes(max_len);
+        cudaError_t e = cudaFuncSetAttribute(topk_rows_bitmap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)bsmem);
+        if (e != cudaSuccess) return e;
+        topk_rows_bitmap_kernel<<<n_rows, kThreads, bsmem, stream>>>(scores, ld, row_begin, row_len, max_len, k, idx,
+                                                                     row_stats);
         return cudaGetLastError();
     }
     const size_t smem = smem_bytes(k);

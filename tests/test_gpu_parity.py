@@ -147,6 +147,51 @@ def test_topk_clustered_near_ties():
         assert np.array_equal(got, oracle.topk(x.astype(np.float64), [n], k))
 
 
+def test_topk_many_long_rows_bit_exact():
+    # At least one row per SM and rows past 16384 entries: the one-CTA-per-row
+    # kernel with the bitmap collect (not the per-row cluster).
+    rng = np.random.default_rng(21)
+    lens = rng.integers(2000, 70000, 160).tolist()
+    lens[:4] = [2049, 16384, 65537, 69999]
+    x = inputs.tie_heavy_scores(len(lens), max(lens), seed=21).numpy()
+    got = gpu_topk(x, 2048, row_len=lens)
+    assert np.array_equal(got, oracle.topk(x.astype(np.float64), lens, 2048))
+
+
+@pytest.mark.parametrize("n_tied", [300, 1000])
+def test_topk_exact_ties_at_the_threshold(n_tied):
+    # 1500 entries above, n_tied entries exactly equal at the k-th value and
+    # the rest below it: the tied entries must be taken lowest index first.
+    # 300 ties are ranked pairwise, 1000 take the whole-row radix path.
+    rng = np.random.default_rng(n_tied)
+    n_rows, n = 150, 20000
+    x = rng.random((n_rows, n), dtype=np.float32)
+    for r in range(n_rows):
+        pos = rng.permutation(n)
+        x[r, pos[:1500]] = 5.0 + rng.random(1500, dtype=np.float32)
+        x[r, pos[1500:1500 + n_tied]] = 3.0
+    got = gpu_topk(x, 2048, row_len=[n] * n_rows)
+    assert np.array_equal(got, oracle.topk(x.astype(np.float64), [n] * n_rows, 2048))
+
+
+def test_topk_rows_beyond_the_bitmap_limit():
+    # A row bound past 557K entries selects the ordered-collect kernel; the
+    # rows themselves are short, so only the bound differs.
+    rng = np.random.default_rng(8)
+    lens = rng.integers(3000, 9000, 150).tolist()
+    x = inputs.tie_heavy_scores(150, max(lens), seed=8).numpy()
+    n_rows, w = x.shape
+    max_len = 600000
+    s = torch.zeros(n_rows, max_len, dtype=torch.float32)
+    s[:, :w] = torch.from_numpy(x)
+    s = s.to(DEV)
+    idx = torch.full((n_rows, 2048), -7, dtype=torch.int32, device=DEV)
+    rl = torch.as_tensor(lens, dtype=torch.int32, device=DEV)
+    dsa.topk(s, 0, n_rows, 2048, idx, row_len=rl, max_len=max_len)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), oracle.topk(x.astype(np.float64), lens, 2048))
+
+
 def test_topk_signed_zeros_and_all_equal():
     x = np.zeros((3, 100), np.float32)
     x[0, ::2] = -0.0
