@@ -20,7 +20,7 @@
 // Keys sit on the MMA M dimension, so the 8-wide N dimension is exactly the
 // 8 heads of a group: no padded rows are multiplied.
 //
-// Prefill: a CTA of 2 warps covers 2 consecutive (query, group) pairs.
+// Prefill: a CTA is one warp, one (query, group) pair.
 // Decode: the k selected rows of a (sequence, group) are split across warps
 // (split-K); each split writes (max, sum, unnormalised O) to the workspace and
 // a combine kernel merges them.
@@ -34,11 +34,13 @@ namespace dsa {
 
 namespace {
 
-// Two stages of 16 keys per warp (16 KB) and two warps per CTA let 14 warps
-// share an SM's shared memory: the kernel is bound by the latency of its L2
-// gathers, so more resident warps (more gathers in flight) beat deeper
-// per-warp pipelines (three stages and 8 warps per SM ran 35 % slower).
-constexpr int kWarpsPerCta = 2;
+// Two stages of 16 keys per warp (16 KB) and one warp per CTA: 13 warps
+// share an SM's shared memory, and a warp's slot is handed to the next
+// (query, group) the moment it finishes, not when its CTA's slowest warp
+// does.  The kernel is bound by the latency of its L2 gathers, so more
+// resident warps beat deeper per-warp pipelines: three stages and 8 warps per
+// SM ran 40 % slower, two warps per CTA 17 % slower.
+constexpr int kWarpsPerCta = 1;
 constexpr int kStages = 2;
 constexpr int kBlk = 16;  // keys per pipeline stage
 
@@ -125,12 +127,15 @@ __device__ __forceinline__ void attend_block(WarpAttn<D> &st, uint32_t ks, uint3
     const float p2 = fast_exp2(s[2] - mref[0]), p3 = fast_exp2(s[3] - mref[1]);
     st.l[0] = st.l[0] * alpha[0] + p0 + p2;
     st.l[1] = st.l[1] * alpha[1] + p1 + p3;
+    // the running max moves on few blocks: skip the rescale when no head's did
+    if (__any_sync(0xFFFFFFFFu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
-    for (int md = 0; md < KT; ++md) {
-        st.o[md][0] *= alpha[0];
-        st.o[md][1] *= alpha[1];
-        st.o[md][2] *= alpha[0];
-        st.o[md][3] *= alpha[1];
+        for (int md = 0; md < KT; ++md) {
+            st.o[md][0] *= alpha[0];
+            st.o[md][1] *= alpha[1];
+            st.o[md][2] *= alpha[0];
+            st.o[md][3] *= alpha[1];
+        }
     }
     // P^T (keys x heads) -> B operand (k = keys, n = heads)
     const uint32_t b0 = movmatrix_trans(pack_bf16x2(p0, p1));
