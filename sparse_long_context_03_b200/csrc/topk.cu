@@ -296,20 +296,17 @@ __device__ void finish_row(TopkSmem &sm, const int32_t *alist, uint32_t cnt, uin
     }
 }
 
-// Threshold bucket of one row (n > k): the value range (from the indexer's
-// row statistics when given), then a histogram over kNB linear buckets of it
-// and the bucket Bt holding the k-th largest entry.  Returns false when the
-// row was finished here (every entry equal, or the exact whole-row path).
-struct RowThreshold {
+// Value range of one row (n > k), from the indexer's row statistics when
+// given, else from a pass over the row; sets the bucket map of the row.
+// Returns false when the row was finished here (every entry equal, or a span
+// that overflows fp32, which takes the exact whole-row path).
+struct RowRange {
     float vmin, scale;
-    uint32_t Bt, need, n_above, cnt;
 };
 
-__device__ bool row_threshold(const float *row, int n, int k, int r, const float *row_stats, TopkSmem &sm,
-                              int32_t *out, RowThreshold &t) {
+__device__ bool row_range(const float *row, int n, int k, int r, const float *row_stats, TopkSmem &sm, int32_t *out,
+                          RowRange &rg) {
     const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
-    float scale;
-    // ---- pass 1: value range (from the indexer's row statistics when given)
     float vmin = INFINITY, vmax = -INFINITY;
     if (row_stats != nullptr) {
         if (tid < 4) {
@@ -338,7 +335,6 @@ __device__ bool row_threshold(const float *row, int n, int k, int r, const float
         fred[warp] = vmin;
         fred[kWarps + warp] = vmax;
     }
-    for (int i = tid; i < kNB; i += kThreads) sm.hist[i] = 0;
     __syncthreads();
     vmin = fred[0];
     vmax = fred[kWarps];
@@ -357,16 +353,32 @@ __device__ bool row_threshold(const float *row, int n, int k, int r, const float
         topk_row_radix(row, n, k, out, sm);
         return false;
     }
+    rg.vmin = vmin;
     // slightly below kNB / range so that vmax itself maps below kNB
-    scale = __fdiv_rn((float)kNB * 0.99999f, range);
+    rg.scale = __fdiv_rn((float)kNB * 0.99999f, range);
+    return true;
+}
 
-    // ---- pass 2: bucket histogram
+// Threshold bucket of one row: a histogram over the kNB buckets of the row's
+// range and the bucket Bt holding the k-th largest entry.  Returns false when
+// the row was finished here (the threshold bucket does not fit in shared
+// memory: exact whole-row path).
+struct RowThreshold {
+    float vmin, scale;
+    uint32_t Bt, need, n_above, cnt;
+};
+
+__device__ bool row_hist_threshold(const float *row, int n, int k, const RowRange &rg, TopkSmem &sm, int32_t *out,
+                                   RowThreshold &t) {
+    const int tid = threadIdx.x;
+    for (int i = tid; i < kNB; i += kThreads) sm.hist[i] = 0;
+    __syncthreads();
     for (int i0 = tid * kVec; i0 < n; i0 += kChunk) {
         float x[kVec];
         const int m = load_vals(row, i0, n, x);
 #pragma unroll
         for (int j = 0; j < kVec; ++j)
-            if (j < m) atomicAdd(&sm.hist[bucket_of(x[j], vmin, scale)], 1u);
+            if (j < m) atomicAdd(&sm.hist[bucket_of(x[j], rg.vmin, rg.scale)], 1u);
     }
     __syncthreads();
     find_threshold_bin(sm.hist, (uint32_t)k, sm.red, sm.bcast);
@@ -375,15 +387,20 @@ __device__ bool row_threshold(const float *row, int n, int k, int r, const float
     t.n_above = sm.bcast[2];    // entries in buckets above it
     t.cnt = sm.hist[t.Bt];
     __syncthreads();
-
     if (t.cnt > (uint32_t)kCap) {
         topk_row_radix(row, n, k, out, sm);
         return false;
     }
-    t.vmin = vmin;
-    t.scale = scale;
+    t.vmin = rg.vmin;
+    t.scale = rg.scale;
     return true;
+}
 
+__device__ bool row_threshold(const float *row, int n, int k, int r, const float *row_stats, TopkSmem &sm,
+                              int32_t *out, RowThreshold &t) {
+    RowRange rg;
+    if (!row_range(row, n, k, r, row_stats, sm, out, rg)) return false;
+    return row_hist_threshold(row, n, k, rg, sm, out, t);
 }
 
 __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__restrict__ scores, int64_t ld,
@@ -450,24 +467,226 @@ __global__ void __launch_bounds__(kThreads) topk_rows_kernel(const float *__rest
 // Many rows of moderate length (prefill chunks): the collect pass marks the
 // selected entries in a bitmap of the row instead of building ordered lists.
 //
-// After the histogram, every entry above the threshold bucket is a winner:
-// its bit is set with one atomicOr per thread and chunk (a thread's kVec = 16
-// entries lie in one 32-bit word).  Threshold-bucket entries go, in any
-// order, to the candidate list through one atomicAdd per warp.  The chosen
-// candidates -- larger key first, then lower index -- set their bits too,
-// and one scan of the bitmap writes the k indices in ascending order.  No
-// block-wide barrier runs inside the pass over the row.  Rows whose tied
-// candidates are too many to rank directly take the whole-row radix path.
+// Threshold band.  With the row's range known in advance (the indexer's row
+// statistics), a histogram of every eighth 16-entry piece of the row brackets
+// the k-th largest entry: the band of buckets [Blo, Bhi] holds the sample's
+// (k f +- m)-th largest entries, f the sampled fraction and m four standard
+// deviations of the sampled count plus four.  Without statistics, or when the
+// band turns out not to contain the k-th entry (or holds too many entries),
+// the full histogram gives the exact threshold bucket (Blo = Bhi = Bt).
+// Either way the selection is exact: the counts that decide it are taken over
+// the whole row in the collect pass, and only the pass that locates the band
+// is sampled.
+//
+// Collect.  Entries above the band are winners: each sets its bit with one
+// atomicOr per thread and chunk (a thread's kVec = 16 entries lie in one
+// 32-bit word).  Entries in the band go, in any order, to the candidate list
+// through one atomicAdd per warp.  No block-wide barrier runs inside the pass.
+// The chosen candidates -- larger key first, then lower index -- set their
+// bits too (a few by direct ranking; more through a second histogram over
+// their own value range), and one scan of the bitmap writes the k indices in
+// ascending order.  Rows whose threshold sub-bucket holds too many entries to
+// rank pairwise (massive exact ties) take the whole-row radix path.
 // ---------------------------------------------------------------------------
 
 constexpr int kMaxTiedRanked = 512;     // tied candidates ranked pairwise
 // Rows up to 524288 entries: the bitmap (64 KB) and the lists still fit twice
 // per SM up to 262144 entries, once beyond.
 constexpr int kBitmapSmemMax = 124 * 1024;
+constexpr int kSampleStride = 8;        // one 16-entry piece in eight is sampled
+// rows of at least 16 k entries are sampled (below that the band's larger
+// candidate list costs about what the skipped histogram saves)
+constexpr int kSampleMinRowPerK = 16;
 
 __host__ __device__ constexpr int bitmap_words(int max_len) { return ((max_len + 31) / 32 + 3) / 4 * 4; }
 __host__ __device__ constexpr size_t bitmap_smem_bytes(int max_len) {
     return sizeof(TopkSmem) + sizeof(uint32_t) * (size_t)bitmap_words(max_len);
+}
+
+// Block-wide sum of one value per thread (two barriers; sm.red reused).
+__device__ __forceinline__ uint32_t block_sum(uint32_t v, TopkSmem &sm) {
+    v = __reduce_add_sync(0xFFFFFFFFu, v);
+    if (lane_id() == 0) sm.red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    uint32_t tot = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) tot += sm.red[w];
+    __syncthreads();
+    return tot;
+}
+
+// One pass over the row: buckets above Bhi set their bits, buckets in
+// [Blo, Bhi] join the candidate list (at most kCap are stored; all are
+// counted).  Returns the number of winners; the candidate count is left in
+// sm.bcast[3].  The trip count is the same for every thread: the warp
+// shuffles need all 32 lanes in every iteration.
+__device__ uint32_t collect_band(const float *row, int n, const RowRange &rg, uint32_t Blo, uint32_t Bhi,
+                                 TopkSmem &sm, uint32_t *bits) {
+    const int tid = threadIdx.x, lane = lane_id();
+    const int words = (n + 31) / 32;
+    for (int w = tid; w < words; w += kThreads) bits[w] = 0u;
+    if (tid == 0) sm.bcast[3] = 0u;
+    __syncthreads();
+    uint32_t n_win = 0;
+    for (int base = 0; base < n; base += kChunk) {
+        const int i0 = base + tid * kVec;
+        float x[kVec] = {};
+        const int m = i0 < n ? load_vals(row, i0, n, x) : 0;
+        uint32_t win = 0u, cmask = 0u;
+#pragma unroll
+        for (int j = 0; j < kVec; ++j) {
+            const uint32_t b = bucket_of(x[j], rg.vmin, rg.scale);
+            if (j < m && b > Bhi) win |= 1u << j;
+            if (j < m && b >= Blo && b <= Bhi) cmask |= 1u << j;
+        }
+        if (win) atomicOr(&bits[i0 >> 5], win << (i0 & 31));
+        n_win += __popc(win);
+        // warp-aggregated slots for the candidates
+        const uint32_t c = __popc(cmask);
+        uint32_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t wtot = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        uint32_t slot = 0u;
+        if (lane == 31 && wtot) slot = atomicAdd(&sm.bcast[3], wtot);
+        slot = __shfl_sync(0xFFFFFFFFu, slot, 31) + incl - c;
+        while (cmask) {
+            const int j = __ffs(cmask) - 1;
+            cmask &= cmask - 1u;
+            if (slot < (uint32_t)kCap) {
+                sm.ckey[slot] = order_key(x[j]);
+                sm.cidx[slot] = i0 + j;
+            }
+            ++slot;
+        }
+    }
+    return block_sum(n_win, sm);  // its barriers also publish the list and the count
+}
+
+// Locate the band from a sample of the row and collect it.  Returns true with
+// the candidate count and the number still to choose when the band holds the
+// k-th largest entry and its candidates fit; false otherwise.
+__device__ bool sampled_band(const float *row, int n, int k, const RowRange &rg, TopkSmem &sm, uint32_t *bits,
+                             uint32_t &cnt, uint32_t &need) {
+    const int tid = threadIdx.x;
+    constexpr int kPiece = kVec * kSampleStride;  // entries from one sampled piece to the next
+    for (int i = tid; i < kNB; i += kThreads) sm.hist[i] = 0;
+    __syncthreads();
+    for (int i0 = tid * kPiece; i0 < n; i0 += kThreads * kPiece) {
+        float x[kVec];
+        const int m = load_vals(row, i0, n, x);
+#pragma unroll
+        for (int j = 0; j < kVec; ++j)
+            if (j < m) atomicAdd(&sm.hist[bucket_of(x[j], rg.vmin, rg.scale)], 1u);
+    }
+    const int pieces = (n + kPiece - 1) / kPiece;
+    const int n_s = (pieces - 1) * kVec + min(kVec, n - (pieces - 1) * kPiece);
+    const float expect = (float)k * (float)n_s / (float)n;
+    const float margin = 4.f * sqrtf(expect) + 4.f;
+    const int need_hi = max(1, (int)floorf(expect - margin));
+    const int need_lo = (int)ceilf(expect + margin);
+    __syncthreads();
+    find_threshold_bin(sm.hist, (uint32_t)need_hi, sm.red, sm.bcast);
+    const uint32_t Bhi = sm.bcast[0];
+    __syncthreads();
+    uint32_t Blo = 0;
+    if (need_lo <= n_s) {
+        find_threshold_bin(sm.hist, (uint32_t)need_lo, sm.red, sm.bcast);
+        Blo = sm.bcast[0];
+        __syncthreads();
+    }
+    const uint32_t n_win = collect_band(row, n, rg, Blo, Bhi, sm, bits);
+    const uint32_t n_cand = sm.bcast[3];
+    __syncthreads();
+    if (n_win > (uint32_t)k || n_win + n_cand < (uint32_t)k || n_cand > (uint32_t)kCap) return false;
+    cnt = n_cand;
+    need = (uint32_t)k - n_win;
+    return true;
+}
+
+// Inverse of order_key (-0.0 comes back as +0.0, which orders the same).
+__device__ __forceinline__ float key_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
+}
+
+// Choose `need` of the cnt candidates (larger key first, lower index on ties)
+// and set their bits: a second histogram over the candidates' own value
+// range finds the sub-bucket holding the need-th largest; entries above it
+// are chosen and the few inside it are ranked pairwise.  Returns false when
+// that sub-bucket holds more than kMaxTiedRanked entries (massive ties): the
+// caller then takes the exact whole-row path.
+__device__ bool choose_by_fine_histogram(TopkSmem &sm, uint32_t *bits, uint32_t cnt, uint32_t need) {
+    if (need == 0) return true;  // the winners alone are the k largest
+    const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
+    float lo = INFINITY, hi = -INFINITY;
+    for (int i = tid; i < (int)cnt; i += kThreads) {
+        const float v = key_value(sm.ckey[i]);
+        lo = fminf(lo, v);
+        hi = fmaxf(hi, v);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+    }
+    float *fred = reinterpret_cast<float *>(sm.red);
+    if (lane == 0) {
+        fred[warp] = lo;
+        fred[kWarps + warp] = hi;
+    }
+    for (int i = tid; i < kNB; i += kThreads) sm.hist[i] = 0;
+    __syncthreads();
+    lo = fred[0];
+    hi = fred[kWarps];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) {
+        lo = fminf(lo, fred[w]);
+        hi = fmaxf(hi, fred[kWarps + w]);
+    }
+    __syncthreads();
+    // equal values: one sub-bucket; otherwise the same monotone map as the row's
+    const float scale = hi > lo ? __fdiv_rn((float)kNB * 0.99999f, hi - lo) : 0.f;
+    for (int i = tid; i < (int)cnt; i += kThreads)
+        atomicAdd(&sm.hist[bucket_of(key_value(sm.ckey[i]), lo, scale)], 1u);
+    __syncthreads();
+    find_threshold_bin(sm.hist, need, sm.red, sm.bcast);
+    const uint32_t Bs = sm.bcast[0];
+    const uint32_t quota = sm.bcast[1];  // to take from sub-bucket Bs
+    const uint32_t in_bs = sm.hist[Bs];
+    __syncthreads();
+    if (in_bs > (uint32_t)kMaxTiedRanked) return false;
+    // entries above Bs are chosen; those in Bs move to a short list (the
+    // histogram's space: 2 x kMaxTiedRanked words) and are ranked there
+    uint32_t *bs_list = sm.hist;
+    if (tid == 0) sm.bcast[3] = 0u;
+    __syncthreads();
+    for (int i = tid; i < (int)cnt; i += kThreads) {
+        const uint32_t ki = sm.ckey[i];
+        const uint32_t b = bucket_of(key_value(ki), lo, scale);
+        if (b > Bs) {
+            const int32_t xi = sm.cidx[i];
+            atomicOr(&bits[xi >> 5], 1u << (xi & 31));
+        } else if (b == Bs) {
+            const uint32_t slot = atomicAdd(&sm.bcast[3], 1u);
+            bs_list[2 * slot] = ki;
+            bs_list[2 * slot + 1] = (uint32_t)sm.cidx[i];
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < (int)in_bs; i += kThreads) {
+        const uint32_t ki = bs_list[2 * i];
+        const int32_t xi = (int32_t)bs_list[2 * i + 1];
+        uint32_t before = 0;  // entries of the sub-bucket that come first
+        for (int j = 0; j < (int)in_bs; ++j) {
+            const uint32_t kj = bs_list[2 * j];
+            before += (kj > ki) || (kj == ki && (int32_t)bs_list[2 * j + 1] < xi);
+        }
+        if (before < quota) atomicOr(&bits[xi >> 5], 1u << (xi & 31));
+    }
+    return true;
 }
 
 __global__ void __launch_bounds__(kThreads) topk_rows_bitmap_kernel(const float *__restrict__ scores, int64_t ld,
@@ -489,51 +708,18 @@ __global__ void __launch_bounds__(kThreads) topk_rows_bitmap_kernel(const float 
         for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
         return;
     }
-    RowThreshold th;
-    if (!row_threshold(row, n, k, r, row_stats, sm, out, th)) return;
-    const uint32_t Bt = th.Bt, need = th.need, cnt = th.cnt;
-
-    const int words = (n + 31) / 32;
-    for (int w = tid; w < words; w += kThreads) bits[w] = 0u;
-    if (tid == 0) sm.bcast[3] = 0u;  // candidates written so far
-    __syncthreads();
-
-    // ---- collect: winners into the bitmap, candidates into the list.  The
-    // trip count is the same for every thread: the warp shuffles below need
-    // all 32 lanes in every iteration.
-    for (int base = 0; base < n; base += kChunk) {
-        const int i0 = base + tid * kVec;
-        float x[kVec] = {};
-        const int m = i0 < n ? load_vals(row, i0, n, x) : 0;
-        uint32_t win = 0u, cmask = 0u;
-#pragma unroll
-        for (int j = 0; j < kVec; ++j) {
-            const uint32_t b = bucket_of(x[j], th.vmin, th.scale);
-            if (j < m && b > Bt) win |= 1u << j;
-            if (j < m && b == Bt) cmask |= 1u << j;
-        }
-        if (win) atomicOr(&bits[i0 >> 5], win << (i0 & 31));
-        // warp-aggregated slots for the candidates
-        const uint32_t c = __popc(cmask);
-        uint32_t incl = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        const uint32_t wtot = __shfl_sync(0xFFFFFFFFu, incl, 31);
-        uint32_t slot = 0u;
-        if (lane == 31 && wtot) slot = atomicAdd(&sm.bcast[3], wtot);
-        slot = __shfl_sync(0xFFFFFFFFu, slot, 31) + incl - c;
-        while (cmask) {
-            const int j = __ffs(cmask) - 1;
-            cmask &= cmask - 1u;
-            sm.ckey[slot] = order_key(x[j]);
-            sm.cidx[slot] = i0 + j;
-            ++slot;
-        }
+    RowRange rg;
+    if (!row_range(row, n, k, r, row_stats, sm, out, rg)) return;
+    uint32_t cnt = 0, need = 0;
+    bool banded = false;
+    if (row_stats != nullptr && n >= kSampleMinRowPerK * k) banded = sampled_band(row, n, k, rg, sm, bits, cnt, need);
+    if (!banded) {
+        RowThreshold th;
+        if (!row_hist_threshold(row, n, k, rg, sm, out, th)) return;
+        (void)collect_band(row, n, rg, th.Bt, th.Bt, sm, bits);
+        cnt = th.cnt;
+        need = th.need;
     }
-    __syncthreads();
 
     // ---- choose `need` of the cnt candidates: larger key first, lower index on ties
     if (cnt <= (uint32_t)kSmallCand) {
@@ -548,38 +734,14 @@ __global__ void __launch_bounds__(kThreads) topk_rows_bitmap_kernel(const float 
             }
             if (rank < need) atomicOr(&bits[xi >> 5], 1u << (xi & 31));
         }
-    } else {
-        uint32_t T, quota;
-        select_in_candidates(sm, (int)cnt, need, T, quota);
-        // how many candidates tie at T
-        uint32_t tied = 0;
-        for (int i = tid; i < (int)cnt; i += kThreads) tied += sm.ckey[i] == T;
-        tied = __reduce_add_sync(0xFFFFFFFFu, tied);
-        if (lane == 0) sm.red[tid >> 5] = tied;
-        __syncthreads();
-        uint32_t n_tied = 0;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) n_tied += sm.red[w];
-        __syncthreads();
-        if (n_tied > (uint32_t)kMaxTiedRanked) {
-            topk_row_radix(row, n, k, out, sm);
-            return;
-        }
-        for (int i = tid; i < (int)cnt; i += kThreads) {
-            const uint32_t ki = sm.ckey[i];
-            const int32_t xi = sm.cidx[i];
-            bool take = ki > T;
-            if (ki == T) {
-                uint32_t before = 0;
-                for (int j = 0; j < (int)cnt; ++j) before += sm.ckey[j] == T && sm.cidx[j] < xi;
-                take = before < quota;
-            }
-            if (take) atomicOr(&bits[xi >> 5], 1u << (xi & 31));
-        }
+    } else if (!choose_by_fine_histogram(sm, bits, cnt, need)) {
+        topk_row_radix(row, n, k, out, sm);
+        return;
     }
     __syncthreads();
 
     // ---- the k set bits, in index order
+    const int words = (n + 31) / 32;
     const int per = (words + kThreads - 1) / kThreads;
     const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
     uint32_t mine = 0;
@@ -594,6 +756,7 @@ __global__ void __launch_bounds__(kThreads) topk_rows_bitmap_kernel(const float 
             out[pos++] = w * 32 + b;
         }
     }
+    (void)lane;
 }
 
 // ---------------------------------------------------------------------------

@@ -192,6 +192,51 @@ def test_topk_rows_beyond_the_bitmap_limit():
     assert np.array_equal(idx.cpu().numpy(), oracle.topk(x.astype(np.float64), lens, 2048))
 
 
+def _gpu_topk_with_stats(x, k, lens):
+    """Top-k with the row statistics the indexer would give (each row's min
+    and max, repeated over the four lane quarters)."""
+    n_rows, w = x.shape
+    ld = (w + 3) // 4 * 4
+    s = torch.zeros(n_rows, ld, dtype=torch.float32)
+    s[:, :w] = torch.from_numpy(x)
+    st = np.zeros((n_rows, 8), np.float32)
+    for r, n in enumerate(lens):
+        st[r, 0::2] = x[r, :n].min()
+        st[r, 1::2] = x[r, :n].max()
+    idx = torch.full((n_rows, k), -7, dtype=torch.int32, device=DEV)
+    dsa.topk(s.to(DEV), 0, n_rows, k, idx, row_len=torch.as_tensor(lens, dtype=torch.int32, device=DEV),
+             max_len=w, row_stats=torch.from_numpy(st).to(DEV))
+    torch.cuda.synchronize()
+    return idx.cpu().numpy()
+
+
+def test_topk_sampled_band_bit_exact():
+    # With row statistics, rows of at least 16 k entries locate their
+    # threshold band from a sample (shorter rows take the full histogram);
+    # the selection must be exact either way.
+    rng = np.random.default_rng(31)
+    lens = rng.integers(16384, 70000, 200).tolist()
+    lens[:3] = [16384, 16385, 69999]
+    x = inputs.tie_heavy_scores(len(lens), max(lens), seed=31).numpy()
+    got = _gpu_topk_with_stats(x, 2048, lens)
+    assert np.array_equal(got, oracle.topk(x.astype(np.float64), lens, 2048))
+
+
+def test_topk_sampled_band_miss_takes_the_exact_path():
+    # The large entries sit only in pieces the sample skips (every eighth
+    # 16-entry piece is sampled), so the band misses the k-th entry; the row
+    # must fall back to the full histogram and give the same exact set.
+    rng = np.random.default_rng(32)
+    n_rows, n = 150, 40000
+    x = rng.random((n_rows, n), dtype=np.float32)
+    unsampled = np.array([i for i in range(n) if (i // 16) % 8 != 0])
+    for r in range(n_rows):
+        pos = rng.choice(unsampled, 3000, replace=False)
+        x[r, pos] = 10.0 + rng.random(3000, dtype=np.float32)
+    got = _gpu_topk_with_stats(x, 2048, [n] * n_rows)
+    assert np.array_equal(got, oracle.topk(x.astype(np.float64), [n] * n_rows, 2048))
+
+
 def test_topk_signed_zeros_and_all_equal():
     x = np.zeros((3, 100), np.float32)
     x[0, ::2] = -0.0
