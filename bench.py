@@ -208,7 +208,7 @@ class PrefillBench:
 TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "dram_traffic.txt")
 STAGE_KERNEL = {"attention": ("sparse_prefill_kernel", "attention.cu"),
                 "indexer": ("indexer_tc_kernel", "indexer_tc.cu"),
-                "topk": ("topk_rows_kernel", "topk.cu")}
+                "topk": ("topk_rows_bitmap_kernel", "topk.cu")}
 
 
 def measured_traffic(stage, workload):
