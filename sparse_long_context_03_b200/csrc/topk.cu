@@ -515,13 +515,13 @@ __device__ __forceinline__ uint32_t block_sum(uint32_t v, TopkSmem &sm) {
     return tot;
 }
 
-// One pass over the row: buckets above Bhi set their bits, buckets in
-// [Blo, Bhi] join the candidate list (at most kCap are stored; all are
+// One pass over the row: entries that classify as winners set their bits,
+// candidates join the candidate list (at most kCap are stored; all are
 // counted).  Returns the number of winners; the candidate count is left in
 // sm.bcast[3].  The trip count is the same for every thread: the warp
 // shuffles need all 32 lanes in every iteration.
-__device__ uint32_t collect_band(const float *row, int n, const RowRange &rg, uint32_t Blo, uint32_t Bhi,
-                                 TopkSmem &sm, uint32_t *bits) {
+template <typename Classify>
+__device__ uint32_t collect_by(const float *row, int n, Classify classify, TopkSmem &sm, uint32_t *bits) {
     const int tid = threadIdx.x, lane = lane_id();
     const int words = (n + 31) / 32;
     for (int w = tid; w < words; w += kThreads) bits[w] = 0u;
@@ -535,9 +535,9 @@ __device__ uint32_t collect_band(const float *row, int n, const RowRange &rg, ui
         uint32_t win = 0u, cmask = 0u;
 #pragma unroll
         for (int j = 0; j < kVec; ++j) {
-            const uint32_t b = bucket_of(x[j], rg.vmin, rg.scale);
-            if (j < m && b > Bhi) win |= 1u << j;
-            if (j < m && b >= Blo && b <= Bhi) cmask |= 1u << j;
+            const uint32_t cls = classify(x[j]);  // 2 winner, 1 candidate, 0 neither
+            if (j < m && cls == 2u) win |= 1u << j;
+            if (j < m && cls == 1u) cmask |= 1u << j;
         }
         if (win) atomicOr(&bits[i0 >> 5], win << (i0 & 31));
         n_win += __popc(win);
@@ -564,6 +564,18 @@ __device__ uint32_t collect_band(const float *row, int n, const RowRange &rg, ui
         }
     }
     return block_sum(n_win, sm);  // its barriers also publish the list and the count
+}
+
+// Collect by buckets: above Bhi winners, [Blo, Bhi] candidates.
+__device__ uint32_t collect_band(const float *row, int n, const RowRange &rg, uint32_t Blo, uint32_t Bhi,
+                                 TopkSmem &sm, uint32_t *bits) {
+    return collect_by(
+        row, n,
+        [&](float x) -> uint32_t {
+            const uint32_t b = bucket_of(x, rg.vmin, rg.scale);
+            return b > Bhi ? 2u : (b >= Blo ? 1u : 0u);
+        },
+        sm, bits);
 }
 
 // Locate the band from a sample of the row and collect it.  Returns true with
@@ -598,7 +610,12 @@ __device__ bool sampled_band(const float *row, int n, int k, const RowRange &rg,
         Blo = sm.bcast[0];
         __syncthreads();
     }
-    const uint32_t n_win = collect_band(row, n, rg, Blo, Bhi, sm, bits);
+    // The pass over the whole row compares values with two thresholds at the
+    // band's bucket edges (any monotone split will do: its counts decide).
+    const float t_hi = rg.vmin + (float)(Bhi + 1) / rg.scale;
+    const float t_lo = Blo == 0 ? -INFINITY : rg.vmin + (float)Blo / rg.scale;
+    const uint32_t n_win = collect_by(
+        row, n, [&](float x) -> uint32_t { return x >= t_hi ? 2u : (x >= t_lo ? 1u : 0u); }, sm, bits);
     const uint32_t n_cand = sm.bcast[3];
     __syncthreads();
     if (n_win > (uint32_t)k || n_win + n_cand < (uint32_t)k || n_cand > (uint32_t)kCap) return false;
