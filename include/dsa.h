@@ -58,7 +58,7 @@ typedef enum {
     DSA_ERR_UNSUPPORTED_SHAPE = 2, /* a head count or head dim this build has no kernel for */
     DSA_ERR_WORKSPACE = 3,         /* workspace missing or smaller than the size query */
     DSA_ERR_CUDA = 4,              /* a kernel launch failed */
-    DSA_ERR_TIMEOUT = 5            /* reserved: a bounded device-side wait gave up */
+    DSA_ERR_TIMEOUT = 5            /* a bounded device-side wait gave up (dsa_check_device_error) */
 } dsa_status_t;
 
 /* Human-readable name of a status code (static storage). */
