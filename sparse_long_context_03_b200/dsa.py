@@ -206,6 +206,40 @@ def prefill_forward(plan: PrefillPlan, q8, sq, w, k8, sk, Q, K, V, O, sm_scale=N
     sparse_gqa_prefill(Q, K, V, plan.idx, 0, plan.L, plan.k, sm_scale, O, lse, stream=stream)
 
 
+def prefill_forward_packed(plan: PrefillPlan, cu_seqlens, q8, sq, w, k8, sk, Q, K, V, O, sm_scale=None, lse=None,
+                           idx_out=None, stream=None):
+    """DSA prefill of several sequences packed along the token axis: sequence
+    b holds tokens cu_seqlens[b] .. cu_seqlens[b+1]-1 (host ints, ascending)
+    and is its own causal prefill -- no query scores or attends a key of
+    another sequence.  Every per-token tensor (q8, sq, w, k8, sk, Q, K, V, O,
+    lse) is indexed by the packed token; the chain runs on each sequence's
+    slice, so `plan` must be sized for the longest sequence.  idx_out, if
+    given, [total, k] int32, receives each token's selected positions within
+    its own sequence."""
+    cu = [int(x) for x in cu_seqlens]
+    if any(b < a for a, b in zip(cu, cu[1:])) or (cu and cu[0] != 0):
+        raise DSAError("cu_seqlens must start at 0 and be non-decreasing")
+    if max((b - a for a, b in zip(cu, cu[1:])), default=0) > plan.L:
+        raise DSAError("a sequence is longer than the plan")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(plan.D)
+    for s0, s1 in zip(cu, cu[1:]):
+        n_tok = s1 - s0
+        if n_tok == 0:
+            continue
+        sl = slice(s0, s1)
+        for r0 in range(0, n_tok, plan.chunk_rows):
+            n = min(plan.chunk_rows, n_tok - r0)
+            indexer_scores(q8[sl], sq[sl], w[sl], k8[sl], sk[sl], r0, n, plan.scores[:n], row_stats=plan.row_stats,
+                           stream=stream)
+            topk(plan.scores[:n], r0, n, plan.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws,
+                 row_stats=plan.row_stats, stream=stream)
+        sparse_gqa_prefill(Q[sl], K[sl], V[sl], plan.idx[:n_tok], 0, n_tok, plan.k, sm_scale, O[sl],
+                           None if lse is None else lse[sl], stream=stream)
+        if idx_out is not None:
+            idx_out[sl].copy_(plan.idx[:n_tok])
+
+
 # ---------------------------------------------------------------------------
 # decode
 # ---------------------------------------------------------------------------

@@ -299,6 +299,60 @@ def test_prefill_chain_tiny_full(use_stats):
     check_attention(O2.float().cpu().numpy(), Oref, l2.cpu().numpy(), lref, "attention on oracle idx")
 
 
+def test_packed_sequences_are_independent_prefills():
+    # Several sequences packed along the token axis: each one is its own
+    # causal prefill.  Compare every token with the oracle run on its own
+    # sequence's slice (empty and one-token sequences included).
+    cfg = inputs.config(0)
+    lens = [300, 1, 0, 777, 64]
+    cu = np.concatenate([[0], np.cumsum(lens)]).tolist()
+    d = inputs.prefill_inputs(cfg, L=cu[-1], seed=41)
+    g = _gpu(d)
+    plan = dsa.PrefillPlan(max(lens), cfg.HI, cfg.dI, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, chunk_rows=256, device=DEV)
+    O = torch.full((cu[-1], cfg.Hq, cfg.D), float("nan"), dtype=torch.bfloat16, device=DEV)
+    lse = torch.full((cu[-1], cfg.Hq), float("nan"), dtype=torch.float32, device=DEV)
+    idx = torch.full((cu[-1], cfg.k), -7, dtype=torch.int32, device=DEV)
+    dsa.prefill_forward_packed(plan, cu, g["q8"], g["sq"], g["w"], g["k8"], g["sk"], g["Q"], g["K"], g["V"], O,
+                               cfg.sm_scale, lse=lse, idx_out=idx)
+    torch.cuda.synchronize()
+    h = {k: H(v) for k, v in d.items()}
+    gidx, Og, lg = idx.cpu().numpy(), O.float().cpu().numpy(), lse.cpu().numpy()
+    for s0, s1 in zip(cu, cu[1:]):
+        if s1 == s0:
+            continue
+        sl = {k: v[s0:s1] for k, v in h.items()}
+        I = oracle.indexer(sl["q8"], sl["sq"], sl["w"], sl["k8"], sl["sk"])
+        ref_idx = oracle.causal_topk(I, 0, cfg.k)
+        for t in range(s1 - s0):
+            check_topk_row(gidx[s0 + t], ref_idx[t], I[t], t + 1, cfg.k, f"sequence at {s0}, row {t}")
+        Oref, lref = oracle.sparse_attention(sl["Q"], sl["K"], sl["V"], ref_idx, 0, cfg.sm_scale)
+        same = np.all(gidx[s0:s1] == ref_idx, axis=1)
+        check_attention(Og[s0:s1][same], Oref[same], lg[s0:s1][same], lref[same], f"sequence at {s0}")
+
+
+def test_prefill_bitwise_deterministic_and_stream_independent():
+    # Same inputs, twice on the default stream and once on a side stream:
+    # indices, outputs and lse must be identical bit for bit (no kernel of
+    # the chain accumulates in a scheduling-dependent order).
+    cfg = inputs.config(1)
+    L = 4096
+    d = _gpu(inputs.prefill_inputs(cfg, L=L, seed=43))
+    runs = []
+    side = torch.cuda.Stream()
+    for stream in (None, None, side):
+        plan = dsa.PrefillPlan(L, cfg.HI, cfg.dI, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, chunk_rows=1500, device=DEV)
+        O = torch.empty(L, cfg.Hq, cfg.D, dtype=torch.bfloat16, device=DEV)
+        lse = torch.empty(L, cfg.Hq, dtype=torch.float32, device=DEV)
+        torch.cuda.synchronize()
+        dsa.prefill_forward(plan, d["q8"], d["sq"], d["w"], d["k8"], d["sk"], d["Q"], d["K"], d["V"], O,
+                            cfg.sm_scale, lse=lse, stream=stream)
+        torch.cuda.synchronize()
+        runs.append((plan.idx.cpu().numpy(), H(O), lse.cpu().numpy()))
+    for other in runs[1:]:
+        for a, b in zip(runs[0], other):
+            assert np.array_equal(a, b)
+
+
 def test_prefill_chain_exact_inputs_bit_exact_indices():
     cfg = inputs.config(1, k=64)
     L = 900
