@@ -11,23 +11,30 @@
 // index order.  No sort, every step is a count, so the result does not
 // depend on scheduling.
 //
-// One CTA owns one row; three passes over the row (the first from HBM, the
-// other two normally from L2):
+// Three kernels share the steps below:
+//   topk_rows_bitmap_kernel   one CTA per row (prefill chunks; row bounds up
+//                             to 557K entries), selection marked in a bitmap;
+//   topk_rows_kernel          one CTA per row for longer row bounds, ordered
+//                             lists;
+//   topk_rows_cluster_kernel  one 8-CTA cluster per row when there are fewer
+//                             rows than SMs (decode).
+// Per row:
 //   1. the row's value range [vmin, vmax] -- skipped when the indexer already
-//      produced it (row statistics), so the histogram pass reads from HBM;
+//      produced it (row statistics);
 //   2. a histogram over 2048 linear buckets of that range (a monotone map,
 //      so bucket order is key order; scores spread over many buckets, which
-//      keeps shared-memory atomics free of hot spots);
-//   3. an ordered collect: entries in buckets above the threshold bucket Bt
-//      are winners, written in index order to a shared list A; entries in Bt
-//      are candidates, written in index order (key, index) to a list C.
+//      keeps shared-memory atomics free of hot spots) -- of the whole row, or,
+//      for long rows with statistics, of a 1/8 sample that brackets the
+//      threshold in a band of buckets (the bitmap kernel; see there);
+//   3. a collect pass: entries above the threshold bucket (or band) are
+//      winners, entries in it are candidates.
 // The chosen candidates (by key, then index) are found by direct ranking when
-// there are few of them, by a small radix select in shared memory otherwise,
-// and compacted in index order; A and the chosen candidates are merged into
-// the output by binary search.  Only candidates are turned into keys.
-// If Bt holds more candidates than fit in shared memory (massive exact ties),
-// the row falls back to a radix select over the whole row (11/11/10-bit
-// passes) followed by an ordered compaction: slower, same result.
+// there are few of them, and otherwise by a small radix select or a second
+// histogram; the output is written in ascending index order.  Only
+// candidates are turned into keys.  If the threshold bucket holds more
+// candidates than fit in shared memory (massive exact ties), the row falls
+// back to a radix select over the whole row (11/11/10-bit passes) followed
+// by an ordered compaction: slower, same result.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -719,7 +726,7 @@ __global__ void __launch_bounds__(kThreads) topk_rows_bitmap_kernel(const float 
     const int n = row_length(row_len, r, row_begin, max_len);
     const float *row = scores + (size_t)r * ld;
     int32_t *out = idx + (size_t)r * k;
-    const int tid = threadIdx.x, lane = lane_id();
+    const int tid = threadIdx.x;
 
     if (n <= k) {  // short row: everything visible is selected
         for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
@@ -773,7 +780,6 @@ __global__ void __launch_bounds__(kThreads) topk_rows_bitmap_kernel(const float 
             out[pos++] = w * 32 + b;
         }
     }
-    (void)lane;
 }
 
 // ---------------------------------------------------------------------------
