@@ -13,9 +13,11 @@
 // registers; the head sum finishes with two xor-shuffles across the 4 lanes
 // that share a key.
 //
-// Two kernels share this: the paged decode indexer (one query per sequence,
-// keys read through the block table) and a prefill fallback used for shapes
-// the tcgen05 kernel does not take.
+// Two kernels share this, both for cases the tcgen05 kernels of
+// indexer_tc.cu do not take: a prefill indexer for HI = 4, and a paged decode
+// indexer (one query per sequence, keys read through the block table) for
+// batches above 4096 sequences.  launch_indexer_decode picks the tcgen05
+// decode kernel whenever it applies.
 #include <type_traits>
 
 #include "common.cuh"
