@@ -3,12 +3,24 @@
 // Host code here only validates arguments, sizes workspaces and launches the
 // kernels on the caller's stream.  It never allocates, frees or synchronises.
 // Validation comes before any CUDA call, so an invalid call touches nothing.
+#include <nvtx3/nvToolsExt.h>
+
 #include <cstring>
 
 #include "dsa.h"
 #include "kernels.h"
 
 namespace {
+
+// One NVTX range per call, named after the entry point, so that a profiler
+// attributes every launch to its stage (header-only NVTX: without a tool
+// attached a range costs a check of a function pointer).
+struct Range {
+    explicit Range(const char *name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+    Range(const Range &) = delete;
+    Range &operator=(const Range &) = delete;
+};
 
 thread_local char g_last_error[256] = "";
 
@@ -72,6 +84,7 @@ size_t dsa_row_stats_bytes(int n_rows) { return n_rows > 0 ? (size_t)n_rows * 8 
 dsa_status_t dsa_indexer_scores(const uint8_t *q8, const float *q_scale, const float *w, const uint8_t *k8,
                                 const float *k_scale, int L, int HI, int dI, int row_begin, int n_rows,
                                 float *scores, int64_t ld_scores, void *row_stats, void *stream) {
+    const Range range(__func__);
     if (L < 1 || row_begin < 0 || n_rows < 0 || (int64_t)row_begin + n_rows > L) return DSA_ERR_INVALID_ARG;
     if (!dsa::indexer_shape_supported(HI, dI)) return DSA_ERR_UNSUPPORTED_SHAPE;
     if (n_rows == 0) return DSA_OK;
@@ -97,6 +110,7 @@ size_t dsa_topk_workspace_size(int n_rows, int max_len, int k) {
 dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, int row_begin, int n_rows, const int32_t *row_len,
                       int max_len, int k, int32_t *idx, const void *row_stats, void *ws, size_t ws_bytes,
                       void *stream) {
+    const Range range(__func__);
     if (n_rows < 0 || row_begin < 0 || k < 1 || max_len < 0) return DSA_ERR_INVALID_ARG;
     if (row_len == nullptr && (int64_t)row_begin + n_rows > max_len) return DSA_ERR_INVALID_ARG;
     if (n_rows == 0) return DSA_OK;
@@ -113,6 +127,7 @@ dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, int row_begin, int
 dsa_status_t dsa_sparse_gqa_prefill(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const int32_t *idx,
                                     int row_begin, int n_rows, int Hq, int Hkv, int D, int k, float sm_scale,
                                     uint16_t *O, float *lse, void *stream) {
+    const Range range(__func__);
     if (row_begin < 0 || n_rows < 0 || k < 1 || Hq < 1 || Hkv < 1) return DSA_ERR_INVALID_ARG;
     if (!dsa::attention_shape_supported(Hq, Hkv, D)) return DSA_ERR_UNSUPPORTED_SHAPE;
     if (n_rows == 0) return DSA_OK;
@@ -140,6 +155,7 @@ dsa_status_t dsa_decode_indexer_scores(const uint8_t *q8, const float *q_scale, 
                                        const int32_t *block_table, int max_pages, int num_pages,
                                        const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI,
                                        float *scores, int64_t ld_scores, void *stream) {
+    const Range range(__func__);
     dsa_status_t st = check_decode_common(block_table, max_pages, num_pages, seq_lens, max_seq_len, B);
     if (st != DSA_OK) return st;
     if (!dsa::indexer_shape_supported(HI, dI)) return DSA_ERR_UNSUPPORTED_SHAPE;
@@ -162,6 +178,7 @@ dsa_status_t dsa_sparse_gqa_decode_attention(const uint16_t *q, const uint16_t *
                                              const int32_t *seq_lens, const int32_t *idx, int B, int Hq, int Hkv,
                                              int D, int k, float sm_scale, void *ws, size_t ws_bytes,
                                              uint16_t *out, float *lse, void *stream) {
+    const Range range(__func__);
     if (B < 0 || k < 1 || Hq < 1 || Hkv < 1 || max_pages < 1 || num_pages < 1) return DSA_ERR_INVALID_ARG;
     if (!dsa::attention_shape_supported(Hq, Hkv, D)) return DSA_ERR_UNSUPPORTED_SHAPE;
     if (B == 0) return DSA_OK;
@@ -179,6 +196,7 @@ dsa_status_t dsa_sparse_gqa_decode_attention_noalloc(const uint16_t *q, const ui
                                                      int max_pages, int num_pages, const int32_t *seq_lens,
                                                      const int32_t *idx, int B, int Hq, int Hkv, int D, int k,
                                                      float sm_scale, uint16_t *out, float *lse, void *stream) {
+    const Range range(__func__);
     if (B < 0 || k < 1 || Hq < 1 || Hkv < 1 || max_pages < 1 || num_pages < 1) return DSA_ERR_INVALID_ARG;
     if (!dsa::attention_shape_supported(Hq, Hkv, D)) return DSA_ERR_UNSUPPORTED_SHAPE;
     if (B == 0) return DSA_OK;
@@ -207,6 +225,7 @@ dsa_status_t dsa_sparse_gqa_decode(const uint16_t *q, const uint8_t *q8, const f
                                    int num_pages, const int32_t *seq_lens, int max_seq_len, int B, int Hq, int Hkv,
                                    int D, int HI, int dI, int k, float sm_scale, void *ws, size_t ws_bytes,
                                    uint16_t *out, int32_t *idx_out, void *stream) {
+    const Range range(__func__);
     dsa_status_t st = check_decode_common(block_table, max_pages, num_pages, seq_lens, max_seq_len, B);
     if (st != DSA_OK) return st;
     if (k < 1 || Hq < 1 || Hkv < 1) return DSA_ERR_INVALID_ARG;
