@@ -103,6 +103,42 @@ def test_decode_rejects_bad_arguments(lib):
     assert call(k=0) == INVALID
 
 
+def test_copies_in_16_byte_pieces_need_aligned_pointers(lib):
+    # TMA boxes and 16-byte copies read these inputs: a pointer off a 16-byte
+    # boundary is rejected before any launch.
+    idx = lib.dsa_indexer_scores
+    assert idx(BOGUS + 4, BOGUS, BOGUS, BOGUS, BOGUS, 512, 4, 32, 0, 8, BOGUS, 512, None, None) == INVALID  # q8
+    assert idx(BOGUS, BOGUS, BOGUS, BOGUS + 8, BOGUS, 512, 4, 32, 0, 8, BOGUS, 512, None, None) == INVALID  # k8
+    dec = lib.dsa_decode_indexer_scores
+
+    def decode_scores(q8=BOGUS, k8c=BOGUS, skc=BOGUS):
+        return dec(q8, BOGUS, BOGUS, k8c, skc, BOGUS, 16, 100, BOGUS, 1000, 4, 32, 64, BOGUS, 1000, None)
+
+    assert decode_scores(q8=BOGUS + 4) == INVALID
+    assert decode_scores(k8c=BOGUS + 16 + 8) == INVALID
+    assert decode_scores(skc=BOGUS + 4) == INVALID
+    chain = lib.dsa_sparse_gqa_decode
+    need = lib.dsa_decode_workspace_size(4, 1000, 32, 4, 128, 64)
+
+    def decode_chain(q8=BOGUS, k8c=BOGUS, skc=BOGUS):
+        return chain(BOGUS, q8, BOGUS, BOGUS, k8c, skc, BOGUS, BOGUS, BOGUS, 16, 100, BOGUS, 1000, 4, 32, 4, 128,
+                     32, 64, 64, 0.1, BOGUS, need, BOGUS, None, None)
+
+    assert decode_chain(q8=BOGUS + 4) == INVALID
+    assert decode_chain(k8c=BOGUS + 4) == INVALID
+    assert decode_chain(skc=BOGUS + 8) == INVALID
+
+
+def test_packed_prefill_rejects_bad_offsets():
+    # checked on the host before any tensor is touched
+    class Plan:
+        L, D = 100, 64
+
+    for cu in ([1, 5], [0, 5, 3], [0, 50, 200]):
+        with pytest.raises(dsa.DSAError):
+            dsa.prefill_forward_packed(Plan(), cu, *([None] * 9), None)
+
+
 def test_workspace_queries(lib):
     a = lib.dsa_decode_workspace_size(32, 262144, 32, 4, 128, 2048)
     b = lib.dsa_decode_workspace_size(32, 131072, 32, 4, 128, 2048)
