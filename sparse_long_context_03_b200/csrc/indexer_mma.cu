@@ -16,8 +16,8 @@
 // Two kernels share this, both for cases the tcgen05 kernels of
 // indexer_tc.cu do not take: a prefill indexer for HI = 4, and a paged decode
 // indexer (one query per sequence, keys read through the block table) for
-// batches above 4096 sequences.  launch_indexer_decode picks the tcgen05
-// decode kernel whenever it applies.
+// batches above 4096 sequences or caches of 2^31 rows and more.
+// launch_indexer_decode picks the tcgen05 decode kernel whenever it applies.
 #include <type_traits>
 
 #include "common.cuh"
@@ -324,8 +324,9 @@ cudaError_t launch_indexer_decode(const uint8_t *q8, const float *sq, const floa
                                   const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI, float *scores,
                                   int64_t ld, cudaStream_t stream) {
     if (B == 0 || max_seq_len == 0) return cudaSuccess;
-    // tensor-core path; this one serves batches beyond its shared-memory prefix
-    if (indexer_decode_tc_supported(HI, dI, B, max_seq_len))
+    // the tensor-core path, unless the batch outgrows its shared-memory prefix
+    // or the cache its 32-bit TMA row coordinates
+    if ((int64_t)num_pages * kPage < (1ll << 31) && indexer_decode_tc_supported(HI, dI, B, max_seq_len))
         return launch_indexer_decode_tc(q8, sq, w, k8c, skc, block_table, max_pages, num_pages, seq_lens, max_seq_len,
                                         B, HI, dI, scores, ld, stream);
     const int pages = (max_seq_len + kPage - 1) / kPage;
