@@ -92,7 +92,8 @@ dsa_status_t dsa_indexer_scores(const uint8_t *q8, const float *q_scale, const f
     if (ld_scores < (int64_t)row_begin + n_rows || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(q8) | reinterpret_cast<uintptr_t>(k8)) % 16 != 0) return DSA_ERR_INVALID_ARG;
     float *stats = static_cast<float *>(row_stats);
-    if (dsa::indexer_tc_supported(HI, dI))
+    // the tensor-core path addresses q8 rows (L * HI of them) with 32-bit TMA coordinates
+    if (dsa::indexer_tc_supported(HI, dI) && (int64_t)L * HI < (1ll << 31))
         return cuda_status(dsa::launch_indexer_prefill_tc(q8, q_scale, w, k8, k_scale, L, HI, dI, row_begin, n_rows,
                                                           scores, ld_scores, stats, as_stream(stream)));
     cudaError_t e = dsa::launch_indexer_prefill_mma(q8, q_scale, w, k8, k_scale, HI, dI, row_begin, n_rows, scores,
