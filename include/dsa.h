@@ -145,7 +145,8 @@ DSA_API dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, int row_be
  *   K, V [>= row_begin + n_rows, Hkv, D] bf16
  *   idx  [n_rows, k] int32 (from dsa_topk)
  *   O    [n_rows, Hq, D] bf16;  lse [n_rows, Hq] float, may be NULL.
- * Supported: D in {64, 128}; Hq % Hkv == 0 with Hq / Hkv <= 8.
+ * Supported: D in {64, 128}; Hq % Hkv == 0 with Hq / Hkv <= 8;
+ * n_rows * Hkv < 2^31 (one CTA per (row, group)).
  * A row with no valid index writes O = 0 and lse = -inf.
  * ------------------------------------------------------------------------ */
 DSA_API dsa_status_t dsa_sparse_gqa_prefill(const uint16_t *Q, const uint16_t *K, const uint16_t *V,

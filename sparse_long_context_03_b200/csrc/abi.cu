@@ -131,6 +131,7 @@ dsa_status_t dsa_sparse_gqa_prefill(const uint16_t *Q, const uint16_t *K, const 
     const Range range(__func__);
     if (row_begin < 0 || n_rows < 0 || k < 1 || Hq < 1 || Hkv < 1) return DSA_ERR_INVALID_ARG;
     if (!dsa::attention_shape_supported(Hq, Hkv, D)) return DSA_ERR_UNSUPPORTED_SHAPE;
+    if ((int64_t)n_rows * Hkv >= (1ll << 31)) return DSA_ERR_UNSUPPORTED_SHAPE;  // one CTA per (row, group)
     if (n_rows == 0) return DSA_OK;
     if (!Q || !K || !V || !idx || !O) return DSA_ERR_INVALID_ARG;
     return cuda_status(dsa::launch_sparse_prefill(Q, K, V, idx, row_begin, n_rows, Hq, Hkv, D, k, sm_scale, O, lse,

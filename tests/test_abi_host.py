@@ -85,6 +85,7 @@ def test_attention_rejects_bad_arguments(lib):
     assert f(BOGUS, BOGUS, BOGUS, BOGUS, 0, 8, 32, 4, 96, 64, 0.1, BOGUS, None, None) == UNSUPPORTED   # D
     assert f(BOGUS, BOGUS, BOGUS, BOGUS, 0, 8, 32, 4, 128, 0, 0.1, BOGUS, None, None) == INVALID
     assert f(None, BOGUS, BOGUS, BOGUS, 0, 8, 32, 4, 128, 64, 0.1, BOGUS, None, None) == INVALID
+    assert f(BOGUS, BOGUS, BOGUS, BOGUS, 0, 2 ** 29, 32, 4, 128, 64, 0.1, BOGUS, None, None) == UNSUPPORTED  # grid
 
 
 def test_decode_rejects_bad_arguments(lib):
