@@ -1,0 +1,52 @@
+"""The benchmark's JSON contract, checked on the host: the reference arm (the
+fp64 oracle timed on the host cores) on the tiny workload, and the lookup of
+recorded DRAM traffic, which must ignore a record whose source no longer
+matches."""
+import hashlib
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+from conftest import ROOT
+
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_reference_arm_prints_the_contract_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "0",
+                          "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["value"] > 0 and line["higher_is_better"] is True
+    assert line["steps"] == 1 and line["warmup"] == 3 and line["n_gpus"] == 1
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_traffic_record_needs_the_current_source(tmp_path, monkeypatch):
+    from sparse_long_context_03_b200 import build
+    src = os.path.join(build.CSRC, "attention.cu")
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    rec = tmp_path / "traffic.txt"
+    rec.write_text("# comment\n"
+                   f"sparse_prefill_kernel prefill-128k 100 20 {digest} attention.cu cmd\n"
+                   f"indexer_tc_kernel prefill-128k 7 8 {'0' * 64} indexer_tc.cu cmd\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(rec))
+    assert bench.measured_traffic("attention", "prefill-128k") == 120
+    assert bench.measured_traffic("attention", "prefill-32k") is None   # other workload
+    assert bench.measured_traffic("indexer", "prefill-128k") is None    # stale hash
+    assert bench.measured_traffic("topk", "prefill-128k") is None       # no record
+
+
+@pytest.mark.parametrize("world", [1, 4])
+def test_weak_scaling_aggregate(world):
+    # whole-job tokens per second: every rank prefills its own sequence
+    assert bench.aggregate_tok_per_s(world, 131072, 5, 500.0) == pytest.approx(world * 131072 * 5 / 0.5)
