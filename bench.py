@@ -30,7 +30,7 @@ import torch  # noqa: E402
 METRIC = "GQA-DSA prefill tok/s @128K & decode step µs; % of HBM / FP8 tensor roofline"
 UNIT = "tok/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-FP8_PER_BF16 = 2.0  # nominal dense ratio, 4.5 / 2.25 PFLOP/s
+FP8_PER_BF16 = 2.0  # nominal dense ratio, 4.5 / 2.25 PFLOP/s (used only if the FP8 measurement fails)
 
 
 def peaks():
@@ -40,6 +40,78 @@ def peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def _best_ms(fn, reps, stream):
+    """Best of `reps` CUDA-event timings of fn() on `stream` (after one warm-up call)."""
+    fn()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(reps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        best = min(best, a.elapsed_time(b))
+    return best
+
+
+def measure_fp8_peak(gpu_index, n=8192, sustain_s=2.0):
+    """Dense FP8 e4m3 GEMM throughput on this GPU: torch._scaled_mm n^3
+    (2 n^3 FLOP), best of 10 (burst) and back to back for ~sustain_s seconds
+    (sustained, under the power cap), with the SM clock sampled meanwhile."""
+    try:
+        a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn).t()  # column-major operand
+        one = torch.ones((), device="cuda", dtype=torch.float32)
+        stream = torch.cuda.current_stream()
+
+        def mm():
+            return torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+
+        burst_ms = _best_ms(mm, 10, stream)
+        with ClockSampler(gpu_index) as clk:
+            iters = max(10, int(sustain_s / (burst_ms / 1e3)))
+            s = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            for _ in range(iters):
+                mm()
+            e.record(stream)
+            torch.cuda.synchronize()
+        sus_ms = s.elapsed_time(e) / iters
+        flop = 2.0 * n ** 3
+        del a, b
+        return {"fp8_tflops": flop / (burst_ms / 1e3) / 1e12, "fp8_tflops_sustained": flop / (sus_ms / 1e3) / 1e12,
+                "how": f"torch._scaled_mm e4m3 x e4m3 -> bf16, {n}^3, best of 10 (burst) and {iters} back to back "
+                       f"(sustained), CUDA events", "clocks_sustained": clk.summary()}
+    except (RuntimeError, TypeError) as exc:  # no FP8 GEMM in this torch build
+        return {"error": str(exc).splitlines()[0][:200]}
+
+
+def measure_read_peaks(dsa):
+    """Read bandwidth of the memory system with the library's read probe
+    (16-byte L2-only loads on every SM): a buffer that fits in L2, read many
+    times (best over a few sizes), and one pass over a 4 GiB buffer (HBM)."""
+    stream = torch.cuda.current_stream()
+    sink = torch.zeros(4, dtype=torch.int32, device="cuda")
+    l2 = {}
+    for mb in (16, 32, 48, 64):
+        buf = torch.ones(mb << 18, dtype=torch.int32, device="cuda")
+        reps = 64
+        ms = _best_ms(lambda: dsa.read_probe(buf, reps, sink), 5, stream)
+        l2[mb] = reps * buf.numel() * 4 / (ms / 1e3) / 1e9
+        del buf
+    big = torch.ones(1 << 30, dtype=torch.int32, device="cuda")
+    ms = _best_ms(lambda: dsa.read_probe(big, 1, sink), 5, stream)
+    hbm_read = big.numel() * 4 / (ms / 1e3) / 1e9
+    del big
+    best_mb = max(l2, key=l2.get)
+    return {"l2_read_gbs": l2[best_mb], "l2_read_gbs_by_mb": l2, "hbm_read_gbs": hbm_read,
+            "how": f"dsa_read_probe: {best_mb} MiB buffer read 64 times (best of 16/32/48/64 MiB, best of 5); "
+                   f"HBM: one pass over 4 GiB, best of 5; CUDA events"}
 
 
 # ----------------------------------------------------------------------------
@@ -101,7 +173,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -147,54 +219,83 @@ def causal_pairs(r0, n):
 
 
 class PrefillBench:
-    def __init__(self, cfg, seed, device, chunk_rows=None):
+    def __init__(self, cfg, seed, device, chunk_rows=None, fused=None):
         from sparse_long_context_03_b200 import dsa, inputs
         self.dsa = dsa
         self.cfg = cfg
         self.d = inputs.prefill_inputs(cfg, device=device, seed=seed)
         self.plan = dsa.PrefillPlan(cfg.L, cfg.HI, cfg.dI, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, chunk_rows=chunk_rows,
-                                    device=device)
+                                    device=device, fused=fused)
         self.O = torch.empty(cfg.L, cfg.Hq, cfg.D, dtype=torch.bfloat16, device=device)
         self.stream = torch.cuda.current_stream()
         self.chunks = list(self.plan.chunks())
+        self.stats = torch.zeros(len(self.chunks), 2, dtype=torch.int64, device=device) if self.plan.fused else None
 
-    def launches_per_step(self):
-        return 2 * len(self.chunks) + 1
+    def stage_names(self):
+        return ["threshold", "indexer", "select", "attention"] if self.plan.fused else ["indexer", "topk", "attention"]
 
     def step(self, ev=None):
         """One whole prefill.  With ev (a dict of lists), brackets every
-        launch with CUDA events on the launching stream."""
+        library call with CUDA events on the launching stream."""
         d, p, c, dsa = self.d, self.plan, self.cfg, self.dsa
-        for r0, n in self.chunks:
-            if ev is not None:
-                a = torch.cuda.Event(enable_timing=True)
-                a.record(self.stream)
-            dsa.indexer_scores(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], r0, n, p.scores[:n], row_stats=p.row_stats)
-            if ev is not None:
-                b = torch.cuda.Event(enable_timing=True)
-                b.record(self.stream)
-            dsa.topk(p.scores[:n], r0, n, c.k, p.idx[r0:r0 + n], max_len=r0 + n, ws=p.ws, row_stats=p.row_stats)
-            if ev is not None:
-                e = torch.cuda.Event(enable_timing=True)
-                e.record(self.stream)
-                ev["indexer"].append((a, b, (r0, n)))
-                ev["topk"].append((b, e, (r0, n)))
-        if ev is not None:
-            a = torch.cuda.Event(enable_timing=True)
-            a.record(self.stream)
+
+        def mark():
+            if ev is None:
+                return None
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(self.stream)
+            return e
+
+        a = mark()
+        for ci, (r0, n) in enumerate(self.chunks):
+            if p.fused:
+                for stage, name in (("threshold", "threshold"), ("candidates", "indexer"), ("select", "select")):
+                    dsa.indexer_topk(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], r0, n, c.k, p.idx[r0:r0 + n], p.ws,
+                                     stats=self.stats[ci] if stage == "select" else None, stage=stage)
+                    b = mark()
+                    if ev is not None:
+                        ev[name].append((a, b, (r0, n)))
+                    a = b
+            else:
+                dsa.indexer_scores(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], r0, n, p.scores[:n],
+                                   row_stats=p.row_stats)
+                b = mark()
+                dsa.topk(p.scores[:n], r0, n, c.k, p.idx[r0:r0 + n], max_len=r0 + n, ws=p.ws, row_stats=p.row_stats)
+                e = mark()
+                if ev is not None:
+                    ev["indexer"].append((a, b, (r0, n)))
+                    ev["topk"].append((b, e, (r0, n)))
+                a = e
         dsa.sparse_gqa_prefill(d["Q"], d["K"], d["V"], p.idx, 0, c.L, c.k, c.sm_scale, self.O)
+        b = mark()
         if ev is not None:
-            b = torch.cuda.Event(enable_timing=True)
-            b.record(self.stream)
             ev["attention"].append((a, b, (0, c.L)))
 
-    # algorithmic work of one launch of each kernel
+    # algorithmic work of one call of each stage
     def flops_indexer(self, r0, n):
+        """4096 FLOP per causal (t, s) pair of the rows that need scores:
+        every row on the unfused path; rows with t + 1 > k on the fused path
+        (a row with t + 1 <= k selects all of 0..t without scoring)."""
         c = self.cfg
+        if self.plan.fused:
+            lo = max(r0, c.k)
+            return 2 * c.HI * c.dI * (causal_pairs(lo, r0 + n - lo) if lo < r0 + n else 0)
         return 2 * c.HI * c.dI * causal_pairs(r0, n)
+
+    def flops_threshold(self, r0, n):
+        """The sampled scores: every 32nd key of the rows scored from candidates."""
+        c = self.cfg
+        keep_all = max(8192, 2 * c.k + 2048)
+        lo = max(r0, keep_all)
+        return 2 * c.HI * c.dI * sum(t // 32 + 1 for t in range(lo, r0 + n))
 
     def bytes_topk(self, r0, n):
         return 4 * causal_pairs(r0, n) + 4 * self.cfg.k * n
+
+    def bytes_select(self, ci, r0, n, cand):
+        """Candidates read (8 B each, counted on the device), 16 B of counts
+        per row, index rows written."""
+        return 8 * cand + 16 * n + 4 * self.cfg.k * n
 
     def bytes_attention(self, r0, n):
         c = self.cfg
@@ -208,7 +309,9 @@ class PrefillBench:
 TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", "dram_traffic.txt")
 STAGE_KERNEL = {"attention": ("sparse_prefill_kernel", "attention.cu"),
                 "indexer": ("indexer_tc_kernel", "indexer_tc.cu"),
-                "topk": ("topk_rows_bitmap_kernel", "topk.cu")}
+                "topk": ("topk_rows_bitmap_kernel", "topk.cu"),
+                "select": ("cand_select_kernel", "topk_fused.cu"),
+                "threshold": ("sample_threshold_kernel", "topk_fused.cu")}
 
 
 def measured_traffic(stage, workload):
@@ -236,7 +339,7 @@ def run_prefill_timed(pb, steps, warmup, world, gpu_index):
     for _ in range(warmup):
         pb.step()
     torch.cuda.synchronize()
-    ev = {"indexer": [], "topk": [], "attention": []}
+    ev = {name: [] for name in pb.stage_names()}
     barrier(world)
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
@@ -358,65 +461,142 @@ class DecodeBench:
         return indexer + scores + gather + small
 
 
-def run_decode_timed(db, steps, warmup):
+def run_decode_timed(db, steps, warmup, gpu_index, min_seconds=0.6):
+    """Decode steps back to back: `steps` of them, or more so that the timed
+    region lasts about min_seconds (long enough for the clock sampler)."""
     for _ in range(warmup):
         db.step()
     torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(db.stream)
+    db.step()
+    b.record(db.stream)
+    torch.cuda.synchronize()
+    steps = max(steps, int(min_seconds * 1e3 / max(a.elapsed_time(b), 1e-3)))
     s = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
-    s.record(db.stream)
-    for _ in range(steps):
-        db.step()
-    e.record(db.stream)
-    torch.cuda.synchronize()
+    with ClockSampler(gpu_index) as clk:
+        s.record(db.stream)
+        for _ in range(steps):
+            db.step()
+        e.record(db.stream)
+        torch.cuda.synchronize()
     db.dsa.check_device_error()
-    return s.elapsed_time(e) / steps
+    return s.elapsed_time(e) / steps, clk.summary()
+
+
+def decode_host_inputs(db):
+    """Host copies of the decode inputs for the oracle, or None when the host
+    has not got twice their size free."""
+    from sparse_long_context_03_b200 import inputs
+    need = sum(v.numel() * v.element_size() for v in db.d.values() if isinstance(v, torch.Tensor))
+    try:
+        import psutil
+        if psutil.virtual_memory().available < 2 * need:
+            return None
+    except ImportError:
+        pass
+    return {k: (inputs.to_numpy_bits(v) if isinstance(v, torch.Tensor) else v) for k, v in db.d.items()}
 
 
 # ----------------------------------------------------------------------------
 # CPU baseline: the fp64 oracle on a bounded sample of the same workload
 # ----------------------------------------------------------------------------
 
-def oracle_prefill_sample(cfg, d_host, n_rows):
-    """Oracle indexer + top-k + attention for n_rows consecutive query rows
-    centred on L/2 (their mean cost equals the whole sequence's mean row cost,
-    since a row's cost grows linearly with t).  Returns (seconds, rows, threads)."""
-    import oracle
-    L = cfg.L
-    r0 = L // 2 - n_rows // 2
-    t0 = time.perf_counter()
-    I = oracle.indexer(d_host["q8"], d_host["sq"], d_host["w"], d_host["k8"], d_host["sk"], row_begin=r0,
-                       n_rows=n_rows)
-    idx = oracle.causal_topk(I, r0, cfg.k)
-    oracle.sparse_attention(d_host["Q_rows"], d_host["K"], d_host["V"], idx, r0, cfg.sm_scale)
-    return time.perf_counter() - t0, n_rows, oracle.threads()
-
-
-def host_inputs_for_oracle(cfg, d, n_rows):
+def sample_rows(cfg, n_total, seed):
+    """Query rows for the oracle: the boundary rows t in {0, k-2, k-1, k,
+    L-1} (plus, on the multimodal workload, the first and last token of a
+    text segment and of the frame after it), then rows drawn uniformly at
+    random without replacement up to n_total."""
+    import numpy as np
     from sparse_long_context_03_b200 import inputs
-    L = cfg.L
-    r0 = L // 2 - n_rows // 2
-    h = {k: inputs.to_numpy_bits(d[k]) for k in ("q8", "sq", "w", "k8", "sk", "K", "V")}
-    h["Q_rows"] = inputs.to_numpy_bits(d["Q"][r0:r0 + n_rows])
-    return h
+    L, k = cfg.L, cfg.k
+    fixed = {0, k - 2, k - 1, k, L - 1}
+    if cfg.multimodal:
+        t0 = inputs.FRAME_TOKENS * inputs.FRAMES_PER_GROUP
+        fixed |= {t0 - 1, t0, t0 + inputs.TEXT_TOKENS - 1, t0 + inputs.TEXT_TOKENS}
+    fixed = sorted(t for t in fixed if 0 <= t < L)
+    rng = np.random.default_rng(seed)
+    pool = np.setdiff1d(np.arange(L), np.asarray(fixed))
+    n_rand = max(0, min(len(pool), n_total - len(fixed)))
+    return sorted(fixed + [int(t) for t in rng.choice(pool, size=n_rand, replace=False)])
 
 
-def cpu_baseline(cfg, d, target_s=15.0):
+def oracle_rows_seconds(cfg, h, rows, threads):
+    """Wall time of the oracle's whole chain (indexer row, top-k, attention)
+    for each query row in `rows`, `threads` rows at a time on the host cores
+    (one oracle thread per row; ctypes releases the GIL during the C call)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+
+    def one(t):
+        oracle.set_threads(1)
+        I = oracle.indexer(h["q8"], h["sq"], h["w"], h["k8"], h["sk"], row_begin=t, n_rows=1)
+        idx = oracle.causal_topk(I, t, cfg.k)
+        oracle.sparse_attention(h["Q"][t:t + 1], h["K"], h["V"], idx, t, cfg.sm_scale)
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(one, rows))
+    return time.perf_counter() - t0
+
+
+def extrapolate_tok_per_s(cfg, rows, seconds):
+    """A row's cost grows with its t+1 visible keys: the whole prefill takes
+    seconds * sum_{t<L}(t+1) / sum_{t in rows}(t+1).  Returns (tok/s, full s)."""
+    units = sum(t + 1 for t in rows)
+    full = seconds * (cfg.L * (cfg.L + 1) / 2) / units
+    return cfg.L / full, full
+
+
+def host_prefill(d):
+    from sparse_long_context_03_b200 import inputs
+    return {k: inputs.to_numpy_bits(d[k]) for k in ("q8", "sq", "w", "k8", "sk", "Q", "K", "V")}
+
+
+def host_cores():
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+
+
+def cpu_baseline(cfg, d, n_rows=256, n_rows_1core=8, decode_host=None, dcfg=None):
+    """The oracle, as it stands, on the host cores: the prefill chain on
+    n_rows sampled rows with every core, and on n_rows_1core of them with one
+    core, each extrapolated to the whole sequence; the decode layer (every
+    sequence, in full) when its host inputs are given."""
     import oracle
     oracle.build()
-    h = host_inputs_for_oracle(cfg, d, 64)
-    n = max(1, oracle.threads())
-    sec, rows, thr = oracle_prefill_sample(cfg, h, n)  # calibration: one row per thread
-    # grow the sample to about target_s seconds of CPU work
-    n2 = int(max(n, min(64, rows * target_s / max(sec, 1e-3))))
-    n2 = max(n, n2 // n * n)
-    if n2 > rows:
-        h = host_inputs_for_oracle(cfg, d, n2)
-        sec, rows, thr = oracle_prefill_sample(cfg, h, n2)
-    return {"value": rows / sec, "unit": UNIT, "cores": thr, "kind": "oracle",
-            "sample": f"{rows} consecutive query rows centred on t=L/2 of the {cfg.L}-token prefill "
-                      f"(whole indexer row, top-k and attention per row, fp64), {sec:.1f} s; "
-                      f"rows/s equals tok/s because their mean cost is the sequence's mean row cost"}
+    h = host_prefill(d)
+    cores = host_cores()
+    rows = sample_rows(cfg, n_rows, seed=cfg.seed)
+    sec = oracle_rows_seconds(cfg, h, rows, cores)
+    value, full = extrapolate_tok_per_s(cfg, rows, sec)
+    # one core: rows spread evenly over the sample
+    sub = rows[:: max(1, len(rows) // n_rows_1core)][:n_rows_1core]
+    sec1 = oracle_rows_seconds(cfg, h, sub, 1)
+    v1, full1 = extrapolate_tok_per_s(cfg, sub, sec1)
+    out = {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+           "sample": f"{len(rows)} query rows of the {cfg.L}-token prefill (t in {{0, k-2, k-1, k, L-1}} and "
+                     f"uniform random rows), whole chain per row (fp64 indexer row, top-k, attention), measured "
+                     f"{sec:.1f} s on {cores} cores; extrapolated to the whole sequence by the per-row cost "
+                     f"sum(t+1): {full:.0f} s",
+           "measured_s": sec, "extrapolated_full_s": full, "rows": len(rows),
+           "one_core": {"value": v1, "unit": UNIT, "cores": 1, "rows": len(sub), "measured_s": sec1,
+                        "extrapolated_full_s": full1}}
+    if decode_host is not None:
+        hd = decode_host
+        oracle.set_threads(cores)
+        t0 = time.perf_counter()
+        Id = oracle.decode_indexer(hd["q8"], hd["sq"], hd["w"], hd["k8_cache"], hd["sk_cache"], hd["block_table"],
+                                   hd["seq_lens"])
+        idx = oracle.topk(Id, hd["seq_lens"], dcfg.k)
+        oracle.decode_attention(hd["q"], hd["k_cache"], hd["v_cache"], hd["block_table"], hd["seq_lens"], idx,
+                                dcfg.sm_scale)
+        dsec = time.perf_counter() - t0
+        out["decode"] = {"step_us": dsec * 1e6, "cores": cores, "higher_is_better": False,
+                         "sample": f"the whole decode step (B={len(hd['seq_lens'])}, every cached token), "
+                                   f"measured, not extrapolated"}
+    return out
 
 
 # ----------------------------------------------------------------------------
@@ -431,25 +611,28 @@ def run_reference(args, rank, world):
     oracle.build()
     cfg = inputs.config(args.config)
     d = inputs.prefill_inputs(cfg, device="cpu", seed=cfg.seed)
-    n = max(1, oracle.threads())
-    h = host_inputs_for_oracle(cfg, d, n)
-    for _ in range(args.warmup):
-        oracle_prefill_sample(cfg, h, n)
-    secs = []
-    for _ in range(args.steps):
-        s, rows, thr = oracle_prefill_sample(cfg, h, n)
-        secs.append(s)
-    total = sum(secs)
-    value = args.steps * n / total
+    h = host_prefill(d)
+    cores = host_cores()
+    per_step = max(cores, 16)
+    for i in range(args.warmup):
+        oracle_rows_seconds(cfg, h, sample_rows(cfg, per_step, seed=cfg.seed + 1 + i), cores)
+    secs, units = 0.0, 0
+    for i in range(args.steps):
+        rows = sample_rows(cfg, per_step, seed=cfg.seed + 1000 + i)
+        secs += oracle_rows_seconds(cfg, h, rows, cores)
+        units += sum(t + 1 for t in rows)
+    full = secs * (cfg.L * (cfg.L + 1) / 2) / units * args.steps  # whole-sequence time of all steps
+    value = args.steps * cfg.L / full
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * full / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"{cfg.name}: DSA prefill L={cfg.L}, Hq={cfg.Hq}, Hkv={cfg.Hkv}, D={cfg.D}, "
                                f"HI={cfg.HI}, dI={cfg.dI}, k={cfg.k}", "seq_len": cfg.L},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
-                         "sample": f"each step: {n} consecutive query rows centred on t=L/2 (fp64 indexer row, "
-                                   f"top-k, attention)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {per_step} query rows (t in {{0, k-2, k-1, k, L-1}} and uniform "
+                                   f"random rows; fp64 indexer row, top-k, attention), measured {secs:.1f} s in "
+                                   f"all, extrapolated to whole sequences by the per-row cost sum(t+1)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -458,9 +641,18 @@ def run_reference(args, rank, world):
 
 # ----------------------------------------------------------------------------
 
-def stage_roofline(per, pb, pk, src):
+def stage_roofline(per, pb, pk, src, fp8, reads):
+    """Per-stage achieved work / time against the stage's own roofline:
+    the indexer against the measured FP8 dense peak, the top-k against the
+    HBM copy peak, the prefill attention against the measured L2 read
+    bandwidth (its gathers are served from L2; its DRAM traffic is far below
+    its algorithmic bytes)."""
     hbm = pk["hbm_gbs"]
-    fp8 = pk["bf16_tflops"] * FP8_PER_BF16
+    if "fp8_tflops" in fp8:
+        fp8_peak, fp8_note = fp8["fp8_tflops"], f"measured FP8 dense (burst): {fp8['how']}"
+    else:
+        fp8_peak = pk["bf16_tflops"] * FP8_PER_BF16
+        fp8_note = f"FP8 measurement failed ({fp8.get('error')}); bf16 burst ({src}) x {FP8_PER_BF16} nominal ratio"
     out = {}
     for name, lst in per.items():
         if not lst:
@@ -469,12 +661,40 @@ def stage_roofline(per, pb, pk, src):
         if name == "indexer":
             work = sum(pb.flops_indexer(*rn) for _, rn in lst)
             ach = work / (tot_ms / 1e3) / 1e12
-            out[name] = {"bound": "tensor", "achieved": ach, "peak": fp8, "unit": "TFLOP/s", "frac": ach / fp8,
+            out[name] = {"bound": "tensor", "achieved": ach, "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": ach / fp8_peak, "ms_total": tot_ms, "launches": len(lst), "peak_note": fp8_note}
+            if "fp8_tflops_sustained" in fp8:
+                out[name]["frac_of_sustained"] = ach / fp8["fp8_tflops_sustained"]
+        elif name == "threshold":
+            work = sum(pb.flops_threshold(*rn) for _, rn in lst)
+            ach = work / (tot_ms / 1e3) / 1e12
+            out[name] = {"bound": "tensor", "achieved": ach, "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": ach / fp8_peak, "ms_total": tot_ms, "launches": len(lst), "peak_note": fp8_note,
+                         "note": "sampled scores (every 32nd key) plus the per-row threshold select over them"}
+        elif name == "select":
+            cand = pb.stats[:, 1].tolist() if pb.stats is not None else [0] * len(lst)
+            steps = max(1, len(lst) // max(1, len(pb.chunks)))
+            work = sum(pb.bytes_select(i % len(pb.chunks), *rn, cand[i % len(pb.chunks)]) for i, (_, rn) in
+                       enumerate(lst))
+            ach = work / (tot_ms / 1e3) / 1e9
+            out[name] = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                         "ms_total": tot_ms, "launches": len(lst), "peak_note": f"HBM copy ({src})",
+                         "candidates_per_row": sum(cand) / pb.cfg.L, "rows_rescored": int(pb.stats[:, 0].sum()),
+                         "note": f"exact top-k of the candidate lists (8 B per candidate read, index rows written); "
+                                 f"{steps} steps"}
+        elif name == "attention":
+            work = sum(pb.bytes_attention(*rn) for _, rn in lst)
+            ach = work / (tot_ms / 1e3) / 1e9
+            l2 = reads["l2_read_gbs"]
+            out[name] = {"bound": "l2", "achieved": ach, "peak": l2, "unit": "GB/s", "frac": ach / l2,
                          "ms_total": tot_ms, "launches": len(lst),
-                         "peak_note": f"FP8 = bf16 burst ({src}) x {FP8_PER_BF16} nominal ratio"}
+                         "peak_note": f"measured L2 read bandwidth ({reads['how']})",
+                         "note": "achieved = algorithmic gather bytes (each selected K/V row once per query and KV "
+                                 "group, plus Q, O and the index rows) / time; the gathers are L2 reads, so the "
+                                 "bound is L2 bandwidth (DRAM traffic per launch is in profiles/)",
+                         "effective_gather_gbs_vs_hbm": ach / hbm}
         else:
-            fn = pb.bytes_topk if name == "topk" else pb.bytes_attention
-            work = sum(fn(*rn) for _, rn in lst)
+            work = sum(pb.bytes_topk(*rn) for _, rn in lst)
             ach = work / (tot_ms / 1e3) / 1e9
             out[name] = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
                          "ms_total": tot_ms, "launches": len(lst), "peak_note": f"HBM copy ({src})"}
@@ -493,6 +713,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--chunk-rows", type=int, default=None,
                     help="query rows per indexer/top-k chunk (default: a 4 GiB score block)")
+    ap.add_argument("--unfused", action="store_true",
+                    help="materialise the score matrix per chunk and run dsa_topk (instead of dsa_indexer_topk)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="sequences in the decode workload (default: the decode-b32 layer's 32)")
     args = ap.parse_args()
@@ -509,39 +731,50 @@ def main():
     barrier(world)
 
     pk, src = peaks()
+    from sparse_long_context_03_b200 import dsa as _dsa
+    fp8, reads = {}, {}
+    if rank == 0:
+        fp8 = measure_fp8_peak(local)
+        reads = measure_read_peaks(_dsa)
+        torch.cuda.empty_cache()
     cfg = inputs.config(args.config)
-    pb = PrefillBench(cfg, seed=rank_seed(cfg, rank), device="cuda", chunk_rows=args.chunk_rows)
+    pb = PrefillBench(cfg, seed=rank_seed(cfg, rank), device="cuda", chunk_rows=args.chunk_rows,
+                      fused=False if args.unfused else None)
     chunk_rows = pb.plan.chunk_rows
+    pb_fused = pb.plan.fused
     ms, per, clocks = run_prefill_timed(pb, args.steps, args.warmup, world, local)
     ms_max = max_over_ranks(ms, world)
     value = aggregate_tok_per_s(world, cfg.L, args.steps, ms_max)
-    stages = stage_roofline(per, pb, pk, src)
-    dominant = max(stages, key=lambda k: stages[k]["ms_total"])
-    dom = dict(stages[dominant])
-    dom_line = {"kernel": dominant, "bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"],
-                "unit": dom["unit"], "frac": dom["frac"], "traffic": measured_traffic(dominant, cfg.name),
-                "peak_source": dom["peak_note"]}
-    if dominant == "attention":
-        dom_line["note"] = ("achieved = algorithmic gather bytes (every selected K/V row once per query and KV "
-                            "group) / time; most rows are served from L2, so it can exceed the HBM copy peak; "
-                            "traffic = DRAM bytes per launch from ncu")
+    stages, dom_line = {}, None
+    if rank == 0:
+        stages = stage_roofline(per, pb, pk, src, fp8, reads)
+        dominant = max(stages, key=lambda k: stages[k]["ms_total"])
+        dom = dict(stages[dominant])
+        dom_line = {"kernel": dominant, "bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"],
+                    "unit": dom["unit"], "frac": dom["frac"], "traffic": measured_traffic(dominant, cfg.name),
+                    "peak_source": dom["peak_note"]}
+        if "note" in dom:
+            dom_line["note"] = dom["note"]
 
     e2e = None
     if not args.no_e2e:
         n_e2e = max(1, args.steps)
-        ems, h2d, d2h = run_prefill_e2e(pb, n_e2e, 1)
+        with ClockSampler(local) as eclk:
+            ems, h2d, d2h = run_prefill_e2e(pb, n_e2e, 1)
         ems = max_over_ranks(ems, world)
         e2e = {"value": aggregate_tok_per_s(world, cfg.L, n_e2e, ems), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ems / n_e2e,
-               "copies": "pinned host buffers; step i+1's inputs up and step i-1's output down during step i"}
+               "copies": "pinned host buffers; step i+1's inputs up and step i-1's output down during step i",
+               "clocks": eclk.summary()}
 
-    decode = None
+    decode, decode_host = None, None
     if not args.no_decode:
         del pb
         torch.cuda.empty_cache()
         dcfg = inputs.config(3)
         db = DecodeBench(dcfg, seed=rank_seed(dcfg, rank), device="cuda", batch=args.decode_batch)
-        us = 1e3 * max_over_ranks(run_decode_timed(db, max(args.steps, 20), max(args.warmup, 3)), world)
+        dms, dclk = run_decode_timed(db, max(args.steps, 20), max(args.warmup, 3), local)
+        us = 1e3 * max_over_ranks(dms, world)
         byts = db.algorithmic_bytes()
         decode = {"workload": f"{dcfg.name}: B={db.B}, cached lengths U[{dcfg.len_lo},{dcfg.len_hi}] "
                               f"(mean {statistics.mean(db.lens):.0f}), page 64, k={dcfg.k}",
@@ -549,13 +782,17 @@ def main():
                   "roofline": {"bound": "hbm", "achieved": byts / (us / 1e6) / 1e9, "peak": pk["hbm_gbs"],
                                "unit": "GB/s", "frac": byts / (us / 1e6) / 1e9 / pk["hbm_gbs"],
                                "algorithmic_bytes": byts},
-                  "gpu_launches_per_step": 4}
+                  "gpu_launches_per_step": 4, "clocks": dclk}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            decode_host = decode_host_inputs(db)
+        del db
+        torch.cuda.empty_cache()
         pb = None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         d_cpu = inputs.prefill_inputs(cfg, device="cuda", seed=cfg.seed)
-        cpu = cpu_baseline(cfg, d_cpu)
+        cpu = cpu_baseline(cfg, d_cpu, decode_host=decode_host, dcfg=inputs.config(3))
         del d_cpu
 
     if rank == 0:
@@ -565,13 +802,20 @@ def main():
             "vs_baseline": None, "dtype": "fp8-e4m3 indexer / bf16 attention (fp32 accumulate)",
             "data": "synthetic (seeded; shapes and distributions of the 128K prefill workload)",
             "config": {"workload": f"{cfg.name}: DSA prefill L={cfg.L}, batch 1 per GPU, Hq={cfg.Hq}, Hkv={cfg.Hkv}, "
-                                   f"D={cfg.D}, HI={cfg.HI}, dI={cfg.dI}, k={cfg.k}, query chunks of {chunk_rows} rows",
+                                   f"D={cfg.D}, HI={cfg.HI}, dI={cfg.dI}, k={cfg.k}, "
+                                   + (f"fused indexer + top-k (no score matrix), query chunks of {chunk_rows} rows"
+                                      if pb_fused else f"score matrix in query chunks of {chunk_rows} rows"),
                        "global_batch": world, "seq_len": cfg.L, "parallelism": f"independent sequences x{world}",
-                       "l2": "inputs larger than L2 (4 GiB score chunks, 1 GiB Q) between launches"},
+                       "l2": "inputs larger than L2 between launches (1 GiB Q and O, 1 GiB of index rows, "
+                             "candidate lists or 4 GiB score chunks)"},
             "roofline": dom_line, "stages": stages, "clocks": clocks, "gpu_launches": None,
+            "peaks_measured_here": {"fp8": fp8, "reads": reads},
             "e2e": e2e, "decode": decode, "cpu_baseline": cpu,
         }
-        line["gpu_launches"] = sum(len(v) for v in per.values())
+        # kernels per library call: the fused threshold stage runs the sampled indexer and the threshold
+        # select, the select stage the candidate select, the repair kernel and the stats copy
+        per_call = {"threshold": 2, "indexer": 1, "select": 3, "topk": 1, "attention": 1}
+        line["gpu_launches"] = sum(per_call[k] * len(v) for k, v in per.items())
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

@@ -131,6 +131,66 @@ DSA_API dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, int row_be
                       const void *row_stats, void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Fused lightning indexer + causal top-k (prefill), one chunk of query rows:
+ * the same Omega_t as dsa_indexer_scores followed by dsa_topk, without
+ * writing the score matrix.
+ *
+ * [REVIEW] 核心公式 (indexer score and Omega_t); [REPORT] 2.3.1; [REPORT]
+ * 5.1.2 (rows with t+1 <= k keep all of 0..t); [REPORT] 5.2.1 (deterministic
+ * top-k; the score matrix is what bounds memory, which the report handles by
+ * chunking -- here it is not materialised at all).
+ * Steps, on `stream`: the indexer scores every 32nd key of each row; a
+ * threshold per row is read off those samples (about 2k keys of a row lie at
+ * or above it); the indexer then scores every causal key and keeps only the
+ * (index, score) pairs at or above the threshold; the exact top-k of those
+ * candidates is taken.  A row whose candidates cannot decide it (fewer than
+ * k of them, or more than fit) is scored again in full and selected exactly,
+ * so the result never depends on the sample: it is the top-k of the row's
+ * fp32 scores, ties to the lower index, -0.0 == +0.0.
+ *
+ *   q8, q_scale, w, k8, k_scale, L, HI, dI, row_begin, n_rows: as for
+ *            dsa_indexer_scores (q8, k8 16-byte aligned; positive scales).
+ *   k        the top-k budget, >= 1.
+ *   idx      [n_rows, k] int32: row r = query t = row_begin + r; ascending,
+ *            -1 padded when t + 1 < k.
+ *   ws       device workspace of dsa_indexer_topk_workspace_size(row_begin,
+ *            n_rows, k, HI, dI) bytes, 256-byte aligned (sampled scores,
+ *            thresholds, candidate lists, the repair list and its scratch
+ *            rows).
+ *   stats    optional (NULL to skip): device int64[2] that receives the
+ *            number of rows of this call that were scored again in full and
+ *            the number of candidates the indexer kept for the selection.
+ * Supported: HI in {8, 16, 32, 64}, dI in {32, 64, 128} (the tensor-core
+ * indexer's shapes), L * HI < 2^31; DSA_ERR_UNSUPPORTED_SHAPE otherwise
+ * (use dsa_indexer_scores + dsa_topk there).
+ * ------------------------------------------------------------------------ */
+DSA_API size_t dsa_indexer_topk_workspace_size(int row_begin, int n_rows, int k, int HI, int dI);
+DSA_API dsa_status_t dsa_indexer_topk(const uint8_t *q8, const float *q_scale, const float *w,
+                              const uint8_t *k8, const float *k_scale,
+                              int L, int HI, int dI, int row_begin, int n_rows, int k,
+                              int32_t *idx, void *ws, size_t ws_bytes, int64_t *stats, void *stream);
+/* The three stages of dsa_indexer_topk, same arguments, for callers that time
+ * or schedule them separately; called in this order on one stream, with the
+ * same workspace and arguments, they are dsa_indexer_topk:
+ *   _threshold   sampled scores (every 32nd key) and one threshold per row;
+ *   _candidates  every causal score, keeping the (index, score) pairs at or
+ *                above the row's threshold (the tensor-core indexer);
+ *   _select      the exact top-k of the candidates into idx, and the full
+ *                re-scoring and selection of any row they cannot decide. */
+DSA_API dsa_status_t dsa_indexer_topk_threshold(const uint8_t *q8, const float *q_scale, const float *w,
+                              const uint8_t *k8, const float *k_scale,
+                              int L, int HI, int dI, int row_begin, int n_rows, int k,
+                              int32_t *idx, void *ws, size_t ws_bytes, int64_t *stats, void *stream);
+DSA_API dsa_status_t dsa_indexer_topk_candidates(const uint8_t *q8, const float *q_scale, const float *w,
+                              const uint8_t *k8, const float *k_scale,
+                              int L, int HI, int dI, int row_begin, int n_rows, int k,
+                              int32_t *idx, void *ws, size_t ws_bytes, int64_t *stats, void *stream);
+DSA_API dsa_status_t dsa_indexer_topk_select(const uint8_t *q8, const float *q_scale, const float *w,
+                              const uint8_t *k8, const float *k_scale,
+                              int L, int HI, int dI, int row_begin, int n_rows, int k,
+                              int32_t *idx, void *ws, size_t ws_bytes, int64_t *stats, void *stream);
+
+/* ------------------------------------------------------------------------
  * Sparse GQA attention (prefill), one chunk of query rows.
  *
  * [REVIEW] 核心公式, u[t,g] = Attn(h[t,g], { c[s,g] | s in Omega_t });
@@ -244,6 +304,21 @@ DSA_API dsa_status_t dsa_sparse_gqa_decode_attention_noalloc(const uint16_t *q,
                                              const int32_t *seq_lens, const int32_t *idx,
                                              int B, int Hq, int Hkv, int D, int k, float sm_scale,
                                              uint16_t *out, float *lse, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Read-bandwidth probe (diagnostic, not part of the layer; the pages have no
+ * counterpart).  Reads `bytes` bytes of `buf` `reps` times with 16-byte loads
+ * cached in L2 only (the load form the attention's gathers use), spread over
+ * every SM, on `stream`.  A caller times it with events: a buffer that fits
+ * in L2 read many times gives the L2 read bandwidth, one pass over a buffer
+ * much larger than L2 gives the HBM read bandwidth; both serve as roofline
+ * denominators.
+ *   buf   device pointer, 16-byte aligned; bytes a multiple of 16, > 0
+ *   sink  device pointer to one uint32 the kernel may write (keeps the
+ *         loads from being optimised away); its value is meaningless
+ *   reps  >= 1
+ * ------------------------------------------------------------------------ */
+DSA_API dsa_status_t dsa_read_probe(const void *buf, size_t bytes, int reps, uint32_t *sink, void *stream);
 
 #ifdef __cplusplus
 }

@@ -125,6 +125,72 @@ dsa_status_t dsa_topk(const float *scores, int64_t ld_scores, int row_begin, int
                                         static_cast<const float *>(row_stats), ws, ws_bytes, as_stream(stream)));
 }
 
+size_t dsa_indexer_topk_workspace_size(int row_begin, int n_rows, int k, int HI, int dI) {
+    if (row_begin < 0 || n_rows < 0 || k < 1 || !dsa::fused_topk_supported(k, HI, dI)) return 0;
+    return dsa::fused_topk_layout(row_begin, n_rows, k, HI, dI).total;
+}
+
+}  // extern "C"
+
+namespace {
+
+dsa_status_t indexer_topk_checked(int stage, const uint8_t *q8, const float *q_scale, const float *w,
+                                  const uint8_t *k8, const float *k_scale, int L, int HI, int dI, int row_begin,
+                                  int n_rows, int k, int32_t *idx, void *ws, size_t ws_bytes, int64_t *stats,
+                                  void *stream) {
+    if (L < 1 || row_begin < 0 || n_rows < 0 || k < 1 || (int64_t)row_begin + n_rows > L) return DSA_ERR_INVALID_ARG;
+    if (!dsa::fused_topk_supported(k, HI, dI) || (int64_t)L * HI >= (1ll << 31)) return DSA_ERR_UNSUPPORTED_SHAPE;
+    if (n_rows == 0) return DSA_OK;
+    if (!q8 || !q_scale || !w || !k8 || !k_scale || !idx) return DSA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(q8) | reinterpret_cast<uintptr_t>(k8)) % 16 != 0) return DSA_ERR_INVALID_ARG;
+    const size_t need = dsa::fused_topk_layout(row_begin, n_rows, k, HI, dI).total;
+    if (ws == nullptr || ws_bytes < need || reinterpret_cast<uintptr_t>(ws) % 256 != 0) return DSA_ERR_WORKSPACE;
+    for (int st = stage == 0 ? 1 : stage; st <= (stage == 0 ? 3 : stage); ++st) {
+        const cudaError_t e = dsa::launch_indexer_topk_stage(st, q8, q_scale, w, k8, k_scale, L, HI, dI, row_begin,
+                                                             n_rows, k, idx, ws, stats, as_stream(stream));
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dsa_status_t dsa_indexer_topk(const uint8_t *q8, const float *q_scale, const float *w, const uint8_t *k8,
+                              const float *k_scale, int L, int HI, int dI, int row_begin, int n_rows, int k,
+                              int32_t *idx, void *ws, size_t ws_bytes, int64_t *stats, void *stream) {
+    const Range range(__func__);
+    return indexer_topk_checked(0, q8, q_scale, w, k8, k_scale, L, HI, dI, row_begin, n_rows, k, idx, ws, ws_bytes,
+                                stats, stream);
+}
+
+dsa_status_t dsa_indexer_topk_threshold(const uint8_t *q8, const float *q_scale, const float *w, const uint8_t *k8,
+                                        const float *k_scale, int L, int HI, int dI, int row_begin, int n_rows,
+                                        int k, int32_t *idx, void *ws, size_t ws_bytes, int64_t *stats,
+                                        void *stream) {
+    const Range range(__func__);
+    return indexer_topk_checked(1, q8, q_scale, w, k8, k_scale, L, HI, dI, row_begin, n_rows, k, idx, ws, ws_bytes,
+                                stats, stream);
+}
+
+dsa_status_t dsa_indexer_topk_candidates(const uint8_t *q8, const float *q_scale, const float *w, const uint8_t *k8,
+                                         const float *k_scale, int L, int HI, int dI, int row_begin, int n_rows,
+                                         int k, int32_t *idx, void *ws, size_t ws_bytes, int64_t *stats,
+                                         void *stream) {
+    const Range range(__func__);
+    return indexer_topk_checked(2, q8, q_scale, w, k8, k_scale, L, HI, dI, row_begin, n_rows, k, idx, ws, ws_bytes,
+                                stats, stream);
+}
+
+dsa_status_t dsa_indexer_topk_select(const uint8_t *q8, const float *q_scale, const float *w, const uint8_t *k8,
+                                     const float *k_scale, int L, int HI, int dI, int row_begin, int n_rows, int k,
+                                     int32_t *idx, void *ws, size_t ws_bytes, int64_t *stats, void *stream) {
+    const Range range(__func__);
+    return indexer_topk_checked(3, q8, q_scale, w, k8, k_scale, L, HI, dI, row_begin, n_rows, k, idx, ws, ws_bytes,
+                                stats, stream);
+}
+
 dsa_status_t dsa_sparse_gqa_prefill(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const int32_t *idx,
                                     int row_begin, int n_rows, int Hq, int Hkv, int D, int k, float sm_scale,
                                     uint16_t *O, float *lse, void *stream) {
@@ -252,6 +318,13 @@ dsa_status_t dsa_sparse_gqa_decode(const uint16_t *q, const uint8_t *q8, const f
     e = dsa::launch_sparse_decode(q, k_cache, v_cache, block_table, max_pages, num_pages, seq_lens, idx, B, Hq, Hkv,
                                   D, k, sm_scale, base + L.attn_off, L.total - L.attn_off, out, nullptr, s);
     return cuda_status(e);
+}
+
+dsa_status_t dsa_read_probe(const void *buf, size_t bytes, int reps, uint32_t *sink, void *stream) {
+    const Range range(__func__);
+    if (!buf || !sink || bytes == 0 || bytes % 16 != 0 || reps < 1) return DSA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(buf) % 16 != 0) return DSA_ERR_INVALID_ARG;
+    return cuda_status(dsa::launch_read_probe(buf, bytes, reps, sink, as_stream(stream)));
 }
 
 }  // extern "C"

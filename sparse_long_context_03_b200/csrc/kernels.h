@@ -25,6 +25,17 @@ cudaError_t launch_indexer_prefill_tc(const uint8_t *q8, const float *sq, const 
                                       const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
                                       float *scores, int64_t ld, float *row_stats, cudaStream_t stream);
 cudaError_t indexer_tc_take_error(unsigned int *flag);
+// the same kernel scoring every indexer_sample_stride()-th key only:
+// sample_scores [n_rows, ld], column j = key j * stride (causal: j * stride <= t)
+int indexer_sample_stride();
+cudaError_t launch_indexer_sample_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
+                                     const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
+                                     float *sample_scores, int64_t ld, cudaStream_t stream);
+// the same kernel keeping only scores >= tau[row]: (index, score) pairs in
+// cand [n_rows, 4, seg_cap], counts (uncapped) in cand_count [n_rows, 4]
+cudaError_t launch_indexer_cand_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
+                                   const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
+                                   const float *tau, int2 *cand, int *cand_count, int seg_cap, cudaStream_t stream);
 bool indexer_decode_tc_supported(int HI, int dI, int B, int max_seq_len);
 cudaError_t launch_indexer_decode_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8c,
                                      const float *skc, const int32_t *block_table, int max_pages, int num_pages,
@@ -37,6 +48,26 @@ bool topk_k_supported(int k);
 cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_rows, const int32_t *row_len,
                         int max_len, int k, int32_t *idx, const float *row_stats, void *ws, size_t ws_bytes,
                         cudaStream_t stream);
+
+// topk_fused.cu: the fused indexer + top-k (sampled threshold, candidate
+// indexer, exact selection of the candidates, repair of undecided rows)
+struct FusedTopkLayout {
+    int keep_all;      // rows with at most this many visible keys keep every key as a candidate
+    int seg_cap;       // candidates per row segment (four segments per row)
+    int64_t lds;       // row stride of the sampled scores
+    int repair_ctas;   // CTAs of the repair kernel (one scratch row each)
+    int64_t scratch_ld;
+    size_t sample_off, tau_off, cand_off, count_off, repair_off, total_off, scratch_off, total;
+    size_t select_smem, repair_smem;
+};
+FusedTopkLayout fused_topk_layout(int row_begin, int n_rows, int k, int HI, int dI);
+bool fused_topk_supported(int k, int HI, int dI);
+// stage 1: sampled scores and per-row thresholds; 2: candidate indexer;
+// 3: exact selection of the candidates and repair of undecided rows
+cudaError_t launch_indexer_topk_stage(int stage, const uint8_t *q8, const float *sq, const float *w,
+                                      const uint8_t *k8, const float *sk, int L, int HI, int dI, int row_begin,
+                                      int n_rows, int k, int32_t *idx, void *ws, int64_t *stats,
+                                      cudaStream_t stream);
 
 // attention.cu
 bool attention_shape_supported(int Hq, int Hkv, int D);
@@ -58,5 +89,9 @@ cudaError_t launch_sparse_decode_fixed_scratch(const uint16_t *q, const uint16_t
                                                const int32_t *seq_lens, const int32_t *idx, int B, int Hq, int Hkv,
                                                int D, int k, float sm_scale, uint16_t *out, float *lse,
                                                cudaStream_t stream);
+
+// probe.cu: streaming 16-byte reads of a buffer, `reps` passes (bandwidth
+// measurement only)
+cudaError_t launch_read_probe(const void *buf, size_t bytes, int reps, uint32_t *sink, cudaStream_t stream);
 
 }  // namespace dsa

@@ -37,6 +37,11 @@ _SIGNATURES = {
     "dsa_indexer_scores": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P, _P], _I),
     "dsa_topk_workspace_size": ([_I, _I, _I], _SZ),
     "dsa_topk": ([_P, _I64, _I, _I, _P, _I, _I, _P, _P, _P, _SZ, _P], _I),
+    "dsa_indexer_topk_workspace_size": ([_I, _I, _I, _I, _I], _SZ),
+    "dsa_indexer_topk": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P, _P], _I),
+    "dsa_indexer_topk_threshold": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P, _P], _I),
+    "dsa_indexer_topk_candidates": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P, _P], _I),
+    "dsa_indexer_topk_select": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P, _P], _I),
     "dsa_sparse_gqa_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P], _I),
     "dsa_decode_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
     "dsa_sparse_gqa_decode": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _I,
@@ -48,6 +53,7 @@ _SIGNATURES = {
     "dsa_decode_attention_fixed_scratch_bytes": ([], _SZ),
     "dsa_sparse_gqa_decode_attention_noalloc": ([_P, _P, _P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _I, _F,
                                                  _P, _P, _P], _I),
+    "dsa_read_probe": ([_P, _SZ, _I, _P, _P], _I),
 }
 
 
@@ -158,6 +164,33 @@ def topk(scores, row_begin, n_rows, k, idx, row_len=None, max_len=None, ws=None,
                           int(k), _ptr(idx), _ptr(row_stats), _ptr(ws), ws_bytes, _stream(stream)), "dsa_topk")
 
 
+def indexer_topk_workspace_size(row_begin, n_rows, k, HI, dI) -> int:
+    return int(lib().dsa_indexer_topk_workspace_size(int(row_begin), int(n_rows), int(k), int(HI), int(dI)))
+
+
+_TOPK_STAGES = {None: "dsa_indexer_topk", "threshold": "dsa_indexer_topk_threshold",
+                "candidates": "dsa_indexer_topk_candidates", "select": "dsa_indexer_topk_select"}
+
+
+def indexer_topk(q8, q_scale, w, k8, k_scale, row_begin, n_rows, k, idx, ws, stats=None, stream=None,
+                 stage=None):
+    """dsa_indexer_topk: Omega_t of query rows [row_begin, row_begin+n_rows)
+    (the top-k of their causal indexer scores, ascending, -1 padded) into
+    idx [n_rows, k] int32, without writing the score matrix.  ``ws`` is a
+    uint8 CUDA tensor of indexer_topk_workspace_size(...) bytes or more;
+    ``stats`` (optional int64 CUDA tensor of 2) receives the number of rows
+    scored again in full and the number of candidates kept.  ``stage`` = "threshold", "candidates" or "select"
+    runs one stage only (dsa_indexer_topk_<stage>)."""
+    _need(q8, torch.uint8, 3, "q8")
+    _need(k8, torch.uint8, 2, "k8")
+    _need(idx, torch.int32, 2, "idx")
+    name = _TOPK_STAGES[stage]
+    L, HI, dI = q8.shape
+    _check(getattr(lib(), name)(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), L, HI, dI,
+                                int(row_begin), int(n_rows), int(k), _ptr(idx), _ptr(ws),
+                                ws.numel() * ws.element_size(), _ptr(stats), _stream(stream)), name)
+
+
 def sparse_gqa_prefill(Q, K, V, idx, row_begin, n_rows, k, sm_scale, O, lse=None, stream=None):
     """dsa_sparse_gqa_prefill: attention of query rows [row_begin, row_begin+n_rows)
     over their selected keys.  Q/O [n_rows,Hq,D] bf16, K/V [L,Hkv,D] bf16."""
@@ -172,37 +205,75 @@ def sparse_gqa_prefill(Q, K, V, idx, row_begin, n_rows, k, sm_scale, O, lse=None
 
 
 class PrefillPlan:
-    """Buffers for a chunked prefill of one sequence (query-row chunks bound
-    the size of the score matrix, as the chunked indexer of report section
-    5.2.1 does).  The score buffer is [chunk_rows, ld] float32."""
+    """Buffers for a prefill of one sequence.
 
-    def __init__(self, L, HI, dI, Hq, Hkv, D, k, chunk_rows=None, device="cuda", score_budget_bytes=4 << 30):
+    fused=True (the default where the shape allows it): the fused indexer +
+    top-k (dsa_indexer_topk), whose workspace holds sampled scores,
+    thresholds and candidate lists instead of the score matrix; query rows
+    are chunked only to keep that workspace within ``fused_budget_bytes``.
+    fused=False: the score matrix of one chunk of query rows at a time
+    ([chunk_rows, ld] float32, the chunked indexer of report section 5.2.1),
+    then dsa_topk."""
+
+    def __init__(self, L, HI, dI, Hq, Hkv, D, k, chunk_rows=None, device="cuda", score_budget_bytes=4 << 30,
+                 fused=None, fused_budget_bytes=24 << 30):
         self.L, self.HI, self.dI, self.Hq, self.Hkv, self.D, self.k = L, HI, dI, Hq, Hkv, D, k
         self.ld = (L + 3) // 4 * 4
-        if chunk_rows is None:
-            chunk_rows = max(1, min(L, score_budget_bytes // (4 * self.ld)))
-        self.chunk_rows = int(chunk_rows)
-        self.scores = torch.empty(self.chunk_rows, self.ld, dtype=torch.float32, device=device)
+        if fused is None:
+            fused = indexer_topk_workspace_size(0, 1, k, HI, dI) > 0
+        self.fused = bool(fused)
         self.idx = torch.empty(L, k, dtype=torch.int32, device=device)
-        need = topk_workspace_size(self.chunk_rows, L, k)
-        self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=device) if need else None
-        self.row_stats = torch.empty(row_stats_bytes(self.chunk_rows), dtype=torch.uint8, device=device)
+        if self.fused:
+            if chunk_rows is None:
+                chunk_rows = L
+                while chunk_rows > 1 and self._fused_ws(chunk_rows) > fused_budget_bytes:
+                    chunk_rows = (chunk_rows + 1) // 2
+            self.chunk_rows = int(chunk_rows)
+            self.scores = None
+            self.row_stats = None
+            self.ws = torch.empty(max(self._fused_ws(self.chunk_rows), 1), dtype=torch.uint8, device=device)
+            self.stats = torch.zeros(2, dtype=torch.int64, device=device)
+        else:
+            if chunk_rows is None:
+                chunk_rows = max(1, min(L, score_budget_bytes // (4 * self.ld)))
+            self.chunk_rows = int(chunk_rows)
+            self.scores = torch.empty(self.chunk_rows, self.ld, dtype=torch.float32, device=device)
+            need = topk_workspace_size(self.chunk_rows, L, k)
+            self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=device) if need else None
+            self.row_stats = torch.empty(row_stats_bytes(self.chunk_rows), dtype=torch.uint8, device=device)
+            self.stats = None
+
+    def _fused_ws(self, chunk_rows):
+        # the workspace grows with the chunk's last row, so the last chunk needs the most
+        need = 0
+        for r0 in range(0, self.L, chunk_rows):
+            need = max(need, indexer_topk_workspace_size(r0, min(chunk_rows, self.L - r0), self.k, self.HI, self.dI))
+        return need
 
     def chunks(self):
         for r0 in range(0, self.L, self.chunk_rows):
             yield r0, min(self.chunk_rows, self.L - r0)
 
 
+def select_rows(plan: PrefillPlan, q8, sq, w, k8, sk, stream=None):
+    """Omega_t of every query row into plan.idx [L, k]: the fused indexer +
+    top-k, or the chunked score matrix followed by dsa_topk."""
+    for r0, n in plan.chunks():
+        if plan.fused:
+            indexer_topk(q8, sq, w, k8, sk, r0, n, plan.k, plan.idx[r0:r0 + n], plan.ws, stream=stream)
+        else:
+            indexer_scores(q8, sq, w, k8, sk, r0, n, plan.scores[:n], row_stats=plan.row_stats, stream=stream)
+            topk(plan.scores[:n], r0, n, plan.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws,
+                 row_stats=plan.row_stats, stream=stream)
+
+
 def prefill_forward(plan: PrefillPlan, q8, sq, w, k8, sk, Q, K, V, O, sm_scale=None, lse=None, stream=None):
-    """Whole DSA prefill of one sequence: for each chunk of query rows, the
-    indexer scores then the top-k; then the sparse attention of every row.
+    """Whole DSA prefill of one sequence: Omega_t of every query row (the
+    indexer and the top-k), then the sparse attention of every row.
     Writes plan.idx [L,k] and O [L,Hq,D] (lse [L,Hq] if given)."""
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(plan.D)
-    for r0, n in plan.chunks():
-        indexer_scores(q8, sq, w, k8, sk, r0, n, plan.scores[:n], row_stats=plan.row_stats, stream=stream)
-        topk(plan.scores[:n], r0, n, plan.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws,
-             row_stats=plan.row_stats, stream=stream)
+    select_rows(plan, q8, sq, w, k8, sk, stream=stream)
     sparse_gqa_prefill(Q, K, V, plan.idx, 0, plan.L, plan.k, sm_scale, O, lse, stream=stream)
 
 
@@ -230,10 +301,14 @@ def prefill_forward_packed(plan: PrefillPlan, cu_seqlens, q8, sq, w, k8, sk, Q, 
         sl = slice(s0, s1)
         for r0 in range(0, n_tok, plan.chunk_rows):
             n = min(plan.chunk_rows, n_tok - r0)
-            indexer_scores(q8[sl], sq[sl], w[sl], k8[sl], sk[sl], r0, n, plan.scores[:n], row_stats=plan.row_stats,
-                           stream=stream)
-            topk(plan.scores[:n], r0, n, plan.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws,
-                 row_stats=plan.row_stats, stream=stream)
+            if plan.fused:
+                indexer_topk(q8[sl], sq[sl], w[sl], k8[sl], sk[sl], r0, n, plan.k, plan.idx[r0:r0 + n], plan.ws,
+                             stream=stream)
+            else:
+                indexer_scores(q8[sl], sq[sl], w[sl], k8[sl], sk[sl], r0, n, plan.scores[:n],
+                               row_stats=plan.row_stats, stream=stream)
+                topk(plan.scores[:n], r0, n, plan.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws,
+                     row_stats=plan.row_stats, stream=stream)
         sparse_gqa_prefill(Q[sl], K[sl], V[sl], plan.idx[:n_tok], 0, n_tok, plan.k, sm_scale, O[sl],
                            None if lse is None else lse[sl], stream=stream)
         if idx_out is not None:
@@ -320,3 +395,18 @@ def sparse_gqa_decode_attention_noalloc(q, k_cache, v_cache, block_table, seq_le
                                                          _ptr(idx), B, Hq, Hkv, D, int(k), float(sm_scale),
                                                          _ptr(out), _ptr(lse), _stream(stream)),
            "dsa_sparse_gqa_decode_attention_noalloc")
+
+
+# ---------------------------------------------------------------------------
+# diagnostics
+# ---------------------------------------------------------------------------
+
+def read_probe(buf, reps, sink, stream=None):
+    """dsa_read_probe: read ``buf`` (a contiguous CUDA tensor, 16-byte
+    multiple) ``reps`` times with L2-only 16-byte loads.  For timing the
+    memory system's read bandwidth; ``sink`` is a small CUDA tensor the kernel
+    may write."""
+    if not buf.is_cuda or not buf.is_contiguous():
+        raise ValueError("buf must be a contiguous CUDA tensor")
+    _check(lib().dsa_read_probe(_ptr(buf), buf.numel() * buf.element_size(), int(reps), _ptr(sink),
+                                _stream(stream)), "dsa_read_probe")

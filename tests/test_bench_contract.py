@@ -50,3 +50,21 @@ def test_traffic_record_needs_the_current_source(tmp_path, monkeypatch):
 def test_weak_scaling_aggregate(world):
     # whole-job tokens per second: every rank prefills its own sequence
     assert bench.aggregate_tok_per_s(world, 131072, 5, 500.0) == pytest.approx(world * 131072 * 5 / 0.5)
+
+
+def test_oracle_sample_rows_and_extrapolation():
+    from sparse_long_context_03_b200 import inputs
+    cfg = inputs.config(2)
+    rows = bench.sample_rows(cfg, 256, seed=5)
+    assert len(rows) == 256 and len(set(rows)) == 256 and rows == sorted(rows)
+    for t in (0, cfg.k - 2, cfg.k - 1, cfg.k, cfg.L - 1):
+        assert t in rows
+    assert all(0 <= t < cfg.L for t in rows)
+    # multimodal: frame/text boundary rows are sampled too
+    mm = inputs.config(4)
+    t0 = inputs.FRAME_TOKENS * inputs.FRAMES_PER_GROUP
+    assert {t0 - 1, t0, t0 + inputs.TEXT_TOKENS - 1, t0 + inputs.TEXT_TOKENS} <= set(bench.sample_rows(mm, 64, 1))
+    # a sample whose rows cost exactly the mean row cost extrapolates by L / n_rows
+    tiny = inputs.config(0, L=9)
+    tok_s, full = bench.extrapolate_tok_per_s(tiny, [4], 2.0)  # mean of t+1 over t<9 is 5
+    assert full == pytest.approx(2.0 * 9) and tok_s == pytest.approx(9 / 18.0)
