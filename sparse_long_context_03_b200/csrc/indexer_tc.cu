@@ -72,6 +72,9 @@ struct EpiShape {
     static constexpr int kMmaWarp = kEpiWarps + 1;  // and kMmaWarp + 1
     static constexpr int kMaxRegs = kThreads > 512 ? 96 : 168;
 };
+// The sampled mode scores every 32nd key (the threshold pre-pass of the
+// fused indexer + top-k).
+constexpr int kSampleStride = 32;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 constexpr uint32_t kIssuerSleepNs = 32;            // back-off of the TMA and MMA warps
 
@@ -96,14 +99,59 @@ struct Layout {
 
 __device__ __forceinline__ void record_timeout() { atomicOr(&g_indexer_tc_error, 1u); }
 
-template <int HI, int DI>
+// What the epilogue does with a score.
+enum IndexerMode : int {
+    kModeScores = 0,   // store every causal score (and optionally each row's range)
+    kModeSample = 1,   // the same over every kSampleStride-th key only (sampled scores)
+    kModeCand = 2,     // keep only scores >= the row's threshold, as (index, score) pairs
+};
+
+// ReLU on the FMA pipe: mul.sat clamps to [0, 1], so with d scaled by 2^-26
+// it returns d * 2^-26 for d >= 0 and 0 otherwise (|d| <= dI * 448^2 < 2^26
+// for e4m3 dot products up to dI = 128; the scaling by a power of two is
+// exact).  The head weight is pre-scaled by 2^26, so w' * y is exactly
+// w * ReLU(d) and the fused multiply-add rounds the same value as the fmax
+// path.  Five head pairs in eight take fmax (ALU pipe), three take mul.sat
+// (FMA pipe), which balances the two pipes against the issue rate.
+constexpr float kSatDown = 1.0f / 67108864.0f;  // 2^-26
+constexpr float kSatUp = 67108864.0f;           // 2^26
+#ifndef DSA_FMAX8
+constexpr int kFmaxPairsPer8 = 5;
+#else
+constexpr int kFmaxPairsPer8 = DSA_FMAX8;  // tuning builds only
+#endif
+__host__ __device__ constexpr bool sat_pair(int p) { return (p & 7) >= kFmaxPairsPer8; }
+
+__device__ __forceinline__ float relu_sat(float d) {
+    float y;
+    asm("mul.rn.sat.f32 %0, %1, %2;\n" : "=f"(y) : "f"(d), "f"(kSatDown));
+    return y;
+}
+
+// Outputs of one launch.  Scores modes: scores [n_rows, ld] (row r = query
+// row_begin + r; in the sampled mode column j is key j * kSampleStride) and
+// optional row_stats [n_rows, 8].  Candidate mode: tau [n_rows] (the row's
+// threshold), cand [n_rows, 4, seg_cap] (index, score) pairs, one segment per
+// TMEM lane quarter, in ascending key order within a segment, and
+// cand_count [n_rows, 4] (the number of entries each segment would hold;
+// entries past seg_cap are dropped).
+struct EpiArgs {
+    float *scores;
+    int64_t ld;
+    float *row_stats;
+    const float *tau;
+    int2 *cand;
+    int *cand_count;
+    int seg_cap;
+};
+
+template <int HI, int DI, int MODE>
 __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                                                  const __grid_constant__ CUtensorMap tmap_q,
                                                                  const float *__restrict__ sq,
                                                                  const float *__restrict__ w,
                                                                  const float *__restrict__ sk, int row_begin,
-                                                                 int n_rows, float *__restrict__ scores,
-                                                                 int64_t ld, float *__restrict__ row_stats) {
+                                                                 int n_rows, const EpiArgs args) {
     using Lay = Layout<DI>;
     using ES = EpiShape<HI>;
     constexpr int kEpiWarps = ES::kEpiWarps, kProducerWarp = ES::kProducerWarp, kMmaWarp = ES::kMmaWarp;
@@ -113,6 +161,8 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
     constexpr int KSTEPS = DI / 32;
     constexpr int kStages = Lay::kStages;
     constexpr uint32_t IDESC = tc::idesc_e4m3_f32(kTileM, kTileN);
+    // key j of the key tensor map is token j * KS; query t sees keys j <= t / KS
+    constexpr int KS = MODE == kModeSample ? kSampleStride : 1;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -171,7 +221,7 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                 const int qb = nb - 1 - i;
                 const int t0 = row_begin + qb * NQ;
                 const int t_hi = min(t0 + NQ, row_end) - 1;
-                const int nstep = t_hi / kStepKeys + 1;
+                const int nstep = (t_hi / KS) / kStepKeys + 1;
                 const int qs = bi & 1;
                 if (!tc::mbar_wait_sleep(qempty_bar(qs), ((bi >> 1) & 1) ^ 1, kWaitLimitNs, kIssuerSleepNs)) {
                     ok = false;
@@ -215,7 +265,7 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                 const int qb = nb - 1 - i;
                 const int t0 = row_begin + qb * NQ;
                 const int t_hi = min(t0 + NQ, row_end) - 1;
-                const int nstep = t_hi / kStepKeys + 1;
+                const int nstep = (t_hi / KS) / kStepKeys + 1;
                 const int qs = bi & 1;
                 if (!tc::mbar_wait_sleep(qfull_bar(qs), (bi >> 1) & 1, kWaitLimitNs, kIssuerSleepNs)) {
                     ok = false;
@@ -258,6 +308,12 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
+        // Thread = one key of the tile (lane quarter qw), CW columns = QPW
+        // whole queries.  (Skipping the causal test on steps that lie wholly
+        // below the block, and the ReLU split between the two pipes, did not
+        // change the time at 128K: with every score stored, the stores and
+        // the math each cost about as much, and the MMA/TMEM pipeline below
+        // them sets a floor about 40 % lower.)
         const int qw = warp & 3;          // TMEM lane quarter: keys 32*qw ..
         const int cg = warp >> 2;         // column group: columns cg*CW ..
         const uint32_t lane_base = tmem_base + ((uint32_t)(qw * 32) << 16);
@@ -267,22 +323,29 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
             const int qb = nb - 1 - i;
             const int t0 = row_begin + qb * NQ;
             const int t_hi = min(t0 + NQ, row_end) - 1;
-            const int nstep = t_hi / kStepKeys + 1;
-            // this warp's query head weights, in registers for the whole block
+            const int nstep = (t_hi / KS) / kStepKeys + 1;
+            // this warp's query head weights, in registers for the whole
+            // block; the pairs that take the mul.sat ReLU are pre-scaled
             float2 wv[CW / 2];
 #pragma unroll
             for (int c = 0; c < CW; c += 2) {
                 const int t = t0 + (cg * CW + c) / HI;
-                wv[c / 2] = t <= t_hi ? __ldg(reinterpret_cast<const float2 *>(w + (size_t)t0 * HI + cg * CW + c))
-                                      : make_float2(0.f, 0.f);
+                float2 x = t <= t_hi ? __ldg(reinterpret_cast<const float2 *>(w + (size_t)t0 * HI + cg * CW + c))
+                                     : make_float2(0.f, 0.f);
+                if (sat_pair(c / 2)) x = make_float2(x.x * kSatUp, x.y * kSatUp);
+                wv[c / 2] = x;
             }
-            float sqv[QPW], vlo[QPW], vhi[QPW];
+            float sqv[QPW], vlo[QPW], vhi[QPW], tau[QPW];
+            int cnt[QPW];
 #pragma unroll
             for (int q = 0; q < QPW; ++q) {
                 const int t = t0 + (cg * CW) / HI + q;
                 sqv[q] = t <= t_hi ? __ldg(sq + t) : 0.f;
                 vlo[q] = INFINITY;
                 vhi[q] = -INFINITY;
+                cnt[q] = 0;
+                if constexpr (MODE == kModeCand) tau[q] = t <= t_hi ? __ldg(args.tau + (t - row_begin)) : INFINITY;
+                else tau[q] = 0.f;
             }
             for (int st = 0; st < nstep; ++st, ++it) {
                 const int pr = it % kPairs;
@@ -291,8 +354,8 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int buf = 2 * pr + h;
-                    const int s = st * kStepKeys + h * kTileM + qw * 32 + lane;
-                    const float sks = s <= t_hi ? __ldg(sk + s) : 0.f;
+                    const int s = st * kStepKeys + h * kTileM + qw * 32 + lane;  // key index (token s * KS)
+                    const float sks = s * KS <= t_hi ? __ldg(sk + (size_t)s * KS) : 0.f;
                     float2 part[QPW][2];
 #pragma unroll
                     for (int q = 0; q < QPW; ++q) part[q][0] = part[q][1] = make_float2(0.f, 0.f);
@@ -311,28 +374,54 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                             const int col = c * 32 + j;              // within this warp's CW columns
                             const int q = col / HI;                  // compile-time after unrolling
                             const int chain = (j >> 2) & 1;
-                            part[q][chain] = tc::ffma2(wv[col / 2],
-                                                       make_float2(fmaxf(acc[j], 0.f), fmaxf(acc[j + 1], 0.f)),
-                                                       part[q][chain]);
-                            part[q][chain] = tc::ffma2(wv[col / 2 + 1],
-                                                       make_float2(fmaxf(acc[j + 2], 0.f), fmaxf(acc[j + 3], 0.f)),
-                                                       part[q][chain]);
+                            const float2 r0 = sat_pair(col / 2)
+                                                  ? make_float2(relu_sat(acc[j]), relu_sat(acc[j + 1]))
+                                                  : make_float2(fmaxf(acc[j], 0.f), fmaxf(acc[j + 1], 0.f));
+                            part[q][chain] = tc::ffma2(wv[col / 2], r0, part[q][chain]);
+                            const float2 r1 = sat_pair(col / 2 + 1)
+                                                  ? make_float2(relu_sat(acc[j + 2]), relu_sat(acc[j + 3]))
+                                                  : make_float2(fmaxf(acc[j + 2], 0.f), fmaxf(acc[j + 3], 0.f));
+                            part[q][chain] = tc::ffma2(wv[col / 2 + 1], r1, part[q][chain]);
                         }
                     }
 #pragma unroll
                     for (int q = 0; q < QPW; ++q) {
                         const int t = t0 + (cg * CW) / HI + q;
-                        if (t <= t_hi && s <= t) {
+                        const bool vis = t <= t_hi && s * KS <= t;
+                        if constexpr (MODE == kModeCand) {
+                            // keep the scores at or above the row's threshold: warp-aggregated
+                            // slots in this warp's own segment of the row (keys in ascending order)
                             const float v = (part[q][0].x + part[q][1].x) + (part[q][0].y + part[q][1].y);
                             const float score = v * sqv[q] * sks;
-                            scores[(size_t)(t - row_begin) * ld + s] = score;
-                            vlo[q] = fminf(vlo[q], score);
-                            vhi[q] = fmaxf(vhi[q], score);
+                            const bool keep = vis && score >= tau[q];
+                            const uint32_t b = __ballot_sync(0xFFFFFFFFu, keep);
+                            if (b != 0u) {
+                                const int pos = cnt[q] + __popc(b & ((1u << lane) - 1u));
+                                if (keep && pos < args.seg_cap)
+                                    args.cand[((size_t)(t - row_begin) * 4 + qw) * args.seg_cap + pos] =
+                                        make_int2(s, __float_as_int(score));
+                                cnt[q] += __popc(b);
+                            }
+                        } else if (vis) {
+                            const float v = (part[q][0].x + part[q][1].x) + (part[q][0].y + part[q][1].y);
+                            const float score = v * sqv[q] * sks;
+                            args.scores[(size_t)(t - row_begin) * args.ld + s] = score;
+                            if constexpr (MODE == kModeScores) {
+                                vlo[q] = fminf(vlo[q], score);
+                                vhi[q] = fmaxf(vhi[q], score);
+                            }
                         }
                     }
                 }
             }
-            if (row_stats != nullptr && ok) {
+            if (!ok) break;
+            if constexpr (MODE == kModeCand) {
+#pragma unroll
+                for (int q = 0; q < QPW; ++q) {
+                    const int t = t0 + (cg * CW) / HI + q;
+                    if (lane == 0 && t <= t_hi) args.cand_count[(size_t)(t - row_begin) * 4 + qw] = cnt[q];
+                }
+            } else if (MODE == kModeScores && args.row_stats != nullptr) {
                 // per-(row, lane quarter) range of the scores just written
 #pragma unroll
                 for (int q = 0; q < QPW; ++q) {
@@ -343,7 +432,7 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                     }
                     const int t = t0 + (cg * CW) / HI + q;
                     if (lane == 0 && t <= t_hi) {
-                        float *st8 = row_stats + (size_t)(t - row_begin) * 8;
+                        float *st8 = args.row_stats + (size_t)(t - row_begin) * 8;
                         st8[2 * qw] = vlo[q];
                         st8[2 * qw + 1] = vhi[q];
                     }
@@ -780,13 +869,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 2D uint8 tensor map: rows of `row_bytes` bytes, boxes of box_rows rows,
-// swizzled by the row width (32/64/128 bytes).
-bool make_map(CUtensorMap *m, const void *base, uint64_t rows, int row_bytes, int box_rows) {
+// 2D uint8 tensor map: rows of `row_bytes` bytes every `row_stride` bytes
+// (row_bytes when 0), boxes of box_rows rows, swizzled by the row width
+// (32/64/128 bytes).
+bool make_map(CUtensorMap *m, const void *base, uint64_t rows, int row_bytes, int box_rows, uint64_t row_stride = 0) {
     auto enc = encode_fn();
     if (enc == nullptr) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    const cuuint64_t strides[1] = {(cuuint64_t)(row_stride ? row_stride : (uint64_t)row_bytes)};
     const cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     const CUtensorMapSwizzle swz = row_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
@@ -804,21 +894,39 @@ int sm_count() {
     return n > 0 ? n : 148;
 }
 
-template <int HI, int DI>
+// Sets a kernel's dynamic shared-memory limit once per device (the
+// attribute is per device and does not change).  One instantiation, and so
+// one set of flags, per kernel.
+template <auto kernel>
+cudaError_t set_smem_once(int smem) {
+    constexpr int kMaxDev = 64;
+    static int done[kMaxDev];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDev && __atomic_load_n(&done[dev], __ATOMIC_ACQUIRE)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess && dev >= 0 && dev < kMaxDev) __atomic_store_n(&done[dev], 1, __ATOMIC_RELEASE);
+    return e;
+}
+
+template <int HI, int DI, int MODE>
 cudaError_t launch_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8, const float *sk, int L,
-                      int row_begin, int n_rows, float *scores, int64_t ld, float *row_stats, cudaStream_t stream) {
+                      int row_begin, int n_rows, const EpiArgs &a, cudaStream_t stream) {
+    constexpr int KS = MODE == kModeSample ? kSampleStride : 1;
     CUtensorMap mk, mq;
-    if (!make_map(&mk, k8, (uint64_t)L, DI, kStepKeys)) return cudaErrorInvalidValue;
+    if (!make_map(&mk, k8, (uint64_t)((L + KS - 1) / KS), DI, kStepKeys, (uint64_t)KS * DI))
+        return cudaErrorInvalidValue;
     if (!make_map(&mq, q8, (uint64_t)L * HI, DI, kTileN)) return cudaErrorInvalidValue;
     constexpr int NQ = kTileN / HI;
     const int nb = (n_rows + NQ - 1) / NQ;
     const int grid = nb < sm_count() ? nb : sm_count();
     // at least 116 KB so that one CTA (and its 512 TMEM columns) owns each SM
     constexpr int smem = Layout<DI>::kAlloc > 116 * 1024 ? Layout<DI>::kAlloc : 116 * 1024;
-    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<HI, DI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_smem_once<indexer_tc_kernel<HI, DI, MODE>>(smem);
     if (e != cudaSuccess) return e;
-    indexer_tc_kernel<HI, DI><<<grid, EpiShape<HI>::kThreads, smem, stream>>>(mk, mq, sq, w, sk, row_begin, n_rows,
-                                                                             scores, ld, row_stats);
+    indexer_tc_kernel<HI, DI, MODE><<<grid, EpiShape<HI>::kThreads, smem, stream>>>(mk, mq, sq, w, sk, row_begin,
+                                                                                   n_rows, a);
     return cudaGetLastError();
 }
 
@@ -843,16 +951,19 @@ bool indexer_tc_supported(int HI, int dI) {
     return (HI == 8 || HI == 16 || HI == 32 || HI == 64) && (dI == 32 || dI == 64 || dI == 128);
 }
 
-cudaError_t launch_indexer_prefill_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
-                                      const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
-                                      float *scores, int64_t ld, float *row_stats, cudaStream_t stream) {
+namespace {
+
+template <int MODE>
+cudaError_t launch_prefill_mode(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
+                                const float *sk, int L, int HI, int dI, int row_begin, int n_rows, const EpiArgs &a,
+                                cudaStream_t stream) {
     if (n_rows == 0) return cudaSuccess;
     auto by_di = [&](auto hi) -> cudaError_t {
         constexpr int H = decltype(hi)::value;
         switch (dI) {
-            case 32: return launch_tc<H, 32>(q8, sq, w, k8, sk, L, row_begin, n_rows, scores, ld, row_stats, stream);
-            case 64: return launch_tc<H, 64>(q8, sq, w, k8, sk, L, row_begin, n_rows, scores, ld, row_stats, stream);
-            case 128: return launch_tc<H, 128>(q8, sq, w, k8, sk, L, row_begin, n_rows, scores, ld, row_stats, stream);
+            case 32: return launch_tc<H, 32, MODE>(q8, sq, w, k8, sk, L, row_begin, n_rows, a, stream);
+            case 64: return launch_tc<H, 64, MODE>(q8, sq, w, k8, sk, L, row_begin, n_rows, a, stream);
+            case 128: return launch_tc<H, 128, MODE>(q8, sq, w, k8, sk, L, row_begin, n_rows, a, stream);
             default: return cudaErrorInvalidValue;
         }
     };
@@ -864,6 +975,40 @@ cudaError_t launch_indexer_prefill_tc(const uint8_t *q8, const float *sq, const 
         default: return cudaErrorInvalidValue;
     }
 }
+
+}  // namespace
+
+cudaError_t launch_indexer_prefill_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
+                                      const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
+                                      float *scores, int64_t ld, float *row_stats, cudaStream_t stream) {
+    EpiArgs a{};
+    a.scores = scores;
+    a.ld = ld;
+    a.row_stats = row_stats;
+    return launch_prefill_mode<kModeScores>(q8, sq, w, k8, sk, L, HI, dI, row_begin, n_rows, a, stream);
+}
+
+cudaError_t launch_indexer_sample_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
+                                     const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
+                                     float *sample_scores, int64_t ld, cudaStream_t stream) {
+    EpiArgs a{};
+    a.scores = sample_scores;
+    a.ld = ld;
+    return launch_prefill_mode<kModeSample>(q8, sq, w, k8, sk, L, HI, dI, row_begin, n_rows, a, stream);
+}
+
+cudaError_t launch_indexer_cand_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
+                                   const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
+                                   const float *tau, int2 *cand, int *cand_count, int seg_cap, cudaStream_t stream) {
+    EpiArgs a{};
+    a.tau = tau;
+    a.cand = cand;
+    a.cand_count = cand_count;
+    a.seg_cap = seg_cap;
+    return launch_prefill_mode<kModeCand>(q8, sq, w, k8, sk, L, HI, dI, row_begin, n_rows, a, stream);
+}
+
+int indexer_sample_stride() { return kSampleStride; }
 
 cudaError_t indexer_tc_take_error(unsigned int *flag) {
     unsigned int zero = 0;

@@ -253,23 +253,34 @@ def test_topk_signed_zeros_and_all_equal():
 # whole prefill chain, small
 # ----------------------------------------------------------------------------
 
-def run_prefill(cfg, d, chunk_rows=None, want_rows=(), lse=True, use_stats=True):
-    """Run the chunked prefill exactly as the benchmark does; also copy out
-    the score rows listed in want_rows as each chunk is produced."""
+def run_prefill(cfg, d, chunk_rows=None, want_rows=(), lse=True, use_stats=True, fused=False):
+    """Run the prefill exactly as the benchmark does (fused=True: the fused
+    indexer + top-k; otherwise the chunked score matrix and dsa_topk); also
+    return the indexer score rows listed in want_rows (the unfused path
+    keeps them as each chunk is produced; the fused path never writes them,
+    so they are scored alone)."""
     L = d["q8"].shape[0]
-    plan = dsa.PrefillPlan(L, cfg.HI, cfg.dI, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, chunk_rows=chunk_rows)
+    plan = dsa.PrefillPlan(L, cfg.HI, cfg.dI, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, chunk_rows=chunk_rows, fused=fused)
     O = torch.empty(L, cfg.Hq, cfg.D, dtype=torch.bfloat16, device=DEV)
     lse_t = torch.empty(L, cfg.Hq, dtype=torch.float32, device=DEV) if lse else None
     want = sorted(want_rows)
     rows = {}
-    for r0, n in plan.chunks():
-        dsa.indexer_scores(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], r0, n, plan.scores[:n],
-                           row_stats=plan.row_stats if use_stats else None)
+    if fused:
+        dsa.select_rows(plan, d["q8"], d["sq"], d["w"], d["k8"], d["sk"])
+        ld = (L + 3) // 4 * 4
+        one = torch.empty(1, ld, dtype=torch.float32, device=DEV)
         for t in want:
-            if r0 <= t < r0 + n:
-                rows[t] = plan.scores[t - r0, : t + 1].cpu().numpy()
-        dsa.topk(plan.scores[:n], r0, n, cfg.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws,
-                 row_stats=plan.row_stats if use_stats else None)
+            dsa.indexer_scores(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], t, 1, one)
+            rows[t] = one[0, : t + 1].cpu().numpy()
+    else:
+        for r0, n in plan.chunks():
+            dsa.indexer_scores(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], r0, n, plan.scores[:n],
+                               row_stats=plan.row_stats if use_stats else None)
+            for t in want:
+                if r0 <= t < r0 + n:
+                    rows[t] = plan.scores[t - r0, : t + 1].cpu().numpy()
+            dsa.topk(plan.scores[:n], r0, n, cfg.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws,
+                     row_stats=plan.row_stats if use_stats else None)
     dsa.sparse_gqa_prefill(d["Q"], d["K"], d["V"], plan.idx, 0, L, cfg.k, cfg.sm_scale, O, lse_t)
     torch.cuda.synchronize()
     return plan, O, lse_t, rows
@@ -578,7 +589,7 @@ def test_full_size_prefill_sampled_rows(cfg_id):
         P = inputs.PERIOD
         extra = [P * 7 + 4095, P * 7 + 4096, P * 7 + 4159, P * 20 + 256]
     rows = _sample_rows(cfg.L, cfg.k, extra, seed=cfg_id)
-    plan, O, lse, got_rows = run_prefill(cfg, d, want_rows=rows)
+    plan, O, lse, got_rows = run_prefill(cfg, d, want_rows=rows, fused=True)
     h = {kk: H(d[kk]) for kk in ("q8", "sq", "w", "k8", "sk")}
     Kh, Vh = H(d["K"]), H(d["V"])
     sel = torch.tensor(rows, device=DEV)
