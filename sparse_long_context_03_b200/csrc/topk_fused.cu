@@ -11,12 +11,12 @@
 // Per chunk of query rows, on one stream:
 //   1. the indexer in its sampled mode scores every 32nd key of each row
 //      (1/32 of the work);
-//   2. sample_threshold_kernel: tau_t = the r-th largest sampled score of
-//      row t, where r is the expected number of sampled keys among the row's
-//      k winners plus seven standard deviations plus eight -- so that, with
-//      overwhelming probability, at least k scores of the row are >= tau_t
-//      and at most a few thousand are.  Rows with at most keep_all visible
-//      keys get tau = -inf (every key is a candidate);
+//   2. sample_threshold_kernel: tau_t = (just below) the r-th largest sampled
+//      score of row t, where r is the expected number of sampled keys among
+//      the row's k winners plus seven standard deviations plus eight -- so
+//      that, with overwhelming probability, at least k scores of the row are
+//      >= tau_t and at most a few thousand are.  Rows with at most keep_all
+//      visible keys get tau = -inf (every key is a candidate);
 //   3. the indexer in its candidate mode computes every causal score and
 //      keeps (index, score) of those >= tau_t, in four segments per row (one
 //      per TMEM lane quarter, each in ascending index order);
@@ -85,30 +85,56 @@ __global__ void __launch_bounds__(kThreads) sample_threshold_kernel(const float 
     }
     const float *row = sample + (size_t)r * lds;
     const bool staged = m <= kStage;
-    if (staged)
-        for (int i = tid; i < m; i += kThreads) sm.ckey[i] = order_key(__ldg(row + i));
-    // rsel-th largest key: three radix passes (11, 11, 10 bits)
-    uint32_t prefix = 0, pmask = 0, need = (uint32_t)rsel;
-#pragma unroll 1
-    for (int p = 0; p < 3; ++p) {
-        const int shift = p == 0 ? 21 : (p == 1 ? 10 : 0);
-        const uint32_t dmask = (p == 2 ? 1023u : 2047u);
-        for (int i = tid; i < kNB; i += kThreads) sm.hist[i] = 0;
+    // The threshold only has to lie at or below the rsel-th largest sample:
+    // the lower edge of the linear bucket (over the samples' range) that
+    // holds it will do, and takes one histogram pass.
+    float lo = INFINITY, hi = -INFINITY;
+    for (int i = tid; i < m; i += kThreads) {
+        const float v = __ldg(row + i);
+        if (staged) sm.ckey[i] = __float_as_uint(v);
+        lo = fminf(lo, v);
+        hi = fmaxf(hi, v);
+    }
+    {
+        const int lane = lane_id(), warp = tid >> 5;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+            hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+        }
+        float *fred = reinterpret_cast<float *>(sm.red);
+        if (lane == 0) {
+            fred[warp] = lo;
+            fred[kWarps + warp] = hi;
+        }
+        for (int b = tid; b < kNB; b += kThreads) sm.hist[b] = 0u;
         __syncthreads();
-        for (int i = tid; i < m; i += kThreads) {
-            const uint32_t key = staged ? sm.ckey[i] : order_key(__ldg(row + i));
-            if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & dmask], 1u);
+        lo = fred[0];
+        hi = fred[kWarps];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) {
+            lo = fminf(lo, fred[w]);
+            hi = fmaxf(hi, fred[kWarps + w]);
         }
         __syncthreads();
-        find_threshold_bin(sm.hist, need, sm.red, sm.bcast);
-        prefix |= sm.bcast[0] << shift;
-        pmask |= dmask << shift;
-        need = sm.bcast[1];
-        __syncthreads();
     }
+    const float range = hi - lo;
+    if (!(range > 0.f && range < INFINITY)) {  // all samples equal (or a span beyond fp32): their minimum
+        if (tid == 0) tau[r] = lo;
+        return;
+    }
+    const float scale = __fdiv_rn((float)kNB * 0.99999f, range);
+    for (int i = tid; i < m; i += kThreads) {
+        const float v = staged ? __uint_as_float(sm.ckey[i]) : __ldg(row + i);
+        atomicAdd(&sm.hist[bucket_of(v, lo, scale)], 1u);
+    }
+    __syncthreads();
+    find_threshold_bin(sm.hist, (uint32_t)rsel, sm.red, sm.bcast);
     if (tid == 0) {
-        const uint32_t key = prefix;
-        tau[r] = __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
+        // bucket B starts at lo + B / scale up to rounding; a hair below it
+        // (only the number of candidates depends on where exactly)
+        const uint32_t B = sm.bcast[0];
+        tau[r] = lo + (float)B * 0.9999f / scale;
     }
 }
 
@@ -121,14 +147,29 @@ struct SelectSmem {
     uint32_t red[2 * kWarps];
     uint32_t bcast[4];
     int seg_off[kSegs + 1];   // candidate slots of segment q: [seg_off[q], seg_off[q+1])
-    int sel_off[kSegs + 1];   // selected entries of segment q: [sel_off[q], sel_off[q+1])
-    uint32_t *ckey;           // [4 * seg_cap] order keys
+    int sel_off[kSegs + 1];   // selected entries of segment q: [sel_off[q], sel_off[q+1]) (merge path)
+    uint32_t *ckey;           // [4 * seg_cap] scores (as bits), then order keys on the radix path
     int32_t *cidx;            // [4 * seg_cap] key indices
-    int32_t *sel;             // [k] selected indices, segment by segment, ascending in each
+    // then, for rows of up to kBitmapMaxN keys, a bitmap of the row's
+    // indices (bit s = key s selected); for longer rows, in the same space,
+    uint32_t *bits;           // [kBitmapMaxN / 32]
+    uint8_t *flag;            // [4 * seg_cap] 1 = selected (merge path)
+    int32_t *sel;             // [k] selected indices, segment by segment, ascending in each (merge path)
 };
 
+// Rows up to this many keys emit their selection through a bitmap of the
+// row (one popcount scan); longer rows merge the four ascending segment
+// lists instead.
+constexpr int kBitmapMaxN = 262144;
+
+__host__ __device__ constexpr size_t select_tail_bytes(int seg_cap, int k) {
+    return (size_t)kBitmapMaxN / 8 > (size_t)kSegs * seg_cap + (size_t)k * 4 + 16
+               ? (size_t)kBitmapMaxN / 8
+               : (size_t)kSegs * seg_cap + (size_t)k * 4 + 16;
+}
+
 __host__ __device__ constexpr size_t select_smem_bytes(int seg_cap, int k) {
-    return (sizeof(SelectSmem) + 15) / 16 * 16 + (size_t)kSegs * seg_cap * 8 + (size_t)k * 4;
+    return (sizeof(SelectSmem) + 15) / 16 * 16 + (size_t)kSegs * seg_cap * 8 + select_tail_bytes(seg_cap, k);
 }
 
 __device__ __forceinline__ void flag_repair(int *repair, int r) {
@@ -161,10 +202,13 @@ __global__ void __launch_bounds__(kThreads) cand_select_kernel(const int2 *__res
         for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
         return;
     }
+    const bool use_bits = n <= kBitmapMaxN;
     if (tid == 0) {
         sm.ckey = reinterpret_cast<uint32_t *>(smem_raw + (sizeof(SelectSmem) + 15) / 16 * 16);
         sm.cidx = reinterpret_cast<int32_t *>(sm.ckey + kSegs * seg_cap);
-        sm.sel = sm.cidx + kSegs * seg_cap;
+        sm.bits = reinterpret_cast<uint32_t *>(sm.cidx + kSegs * seg_cap);
+        sm.sel = reinterpret_cast<int32_t *>(sm.bits);
+        sm.flag = reinterpret_cast<uint8_t *>(sm.sel + k);
         int total = 0;
         bool bad = false;
         sm.seg_off[0] = 0;
@@ -183,55 +227,177 @@ __global__ void __launch_bounds__(kThreads) cand_select_kernel(const int2 *__res
         return;
     }
     const int total = sm.seg_off[kSegs];
-    // load the candidates, segment after segment
+    const int words = (n + 31) / 32;
+    if (use_bits)
+        for (int i = tid; i < words; i += kThreads) sm.bits[i] = 0u;
+    // load the candidates, segment after segment, and their value range
+    // (two candidates per 16-byte load where a segment's start allows it)
+    float lo = INFINITY, hi = -INFINITY;
     for (int q = 0; q < kSegs; ++q) {
         const int2 *src = cand + ((size_t)r * kSegs + q) * seg_cap;
         const int o = sm.seg_off[q], c = sm.seg_off[q + 1] - o;
-        for (int i = tid; i < c; i += kThreads) {
+        const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
+        const int c2 = vec ? c / 2 : 0;
+        for (int i = tid; i < c2; i += kThreads) {
+            const int4 e = __ldg(reinterpret_cast<const int4 *>(src) + i);
+            const float v0 = __int_as_float(e.y), v1 = __int_as_float(e.w);
+            lo = fminf(lo, fminf(v0, v1));
+            hi = fmaxf(hi, fmaxf(v0, v1));
+            sm.ckey[o + 2 * i] = (uint32_t)e.y;
+            sm.cidx[o + 2 * i] = e.x;
+            sm.ckey[o + 2 * i + 1] = (uint32_t)e.w;
+            sm.cidx[o + 2 * i + 1] = e.z;
+        }
+        for (int i = 2 * c2 + tid; i < c; i += kThreads) {
             const int2 e = __ldg(src + i);
-            sm.ckey[o + i] = order_key(__int_as_float(e.y));
+            const float v = __int_as_float(e.y);
+            lo = fminf(lo, v);
+            hi = fmaxf(hi, v);
+            sm.ckey[o + i] = (uint32_t)e.y;
             sm.cidx[o + i] = e.x;
         }
     }
-    __syncthreads();
-    // T = the k-th largest key; quota = how many entries equal to T are taken
-    uint32_t T, quota;
-    select_in_candidates(sm, total, (uint32_t)k, T, quota);
-    const uint32_t tied = sm.hist[T & 1023u];  // the last pass's bin of T holds every entry equal to T
-    __syncthreads();
-    if (tied > (uint32_t)kMaxTies) {
-        if (tid == 0) flag_repair(repair, r);
-        return;
+    {
+        const int lane = lane_id(), warp = tid >> 5;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+            hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+        }
+        float *fred = reinterpret_cast<float *>(sm.red);
+        if (lane == 0) {
+            fred[warp] = lo;
+            fred[kWarps + warp] = hi;
+        }
+        for (int b = tid; b < kNB; b += kThreads) sm.hist[b] = 0u;
+        __syncthreads();
+        lo = fred[0];
+        hi = fred[kWarps];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) {
+            lo = fminf(lo, fred[w]);
+            hi = fmaxf(hi, fred[kWarps + w]);
+        }
+        __syncthreads();
     }
-    // entries equal to T: the quota lowest indices (ranked pairwise in a
-    // short list kept in the histogram's space)
-    uint32_t *tlist = sm.hist;  // [2 * kMaxTies]: (slot, index)
-    if (tied != quota) {
+    // mark(i): candidate in slot i is selected
+    auto mark = [&](int i) {
+        if (use_bits) {
+            const int32_t x = sm.cidx[i];
+            atomicOr(&sm.bits[x >> 5], 1u << (x & 31));
+        } else {
+            sm.flag[i] = 1;
+        }
+    };
+    // Linear buckets over [lo, hi] (a monotone map: bucket order is score
+    // order, equal scores share a bucket): the bucket Bt holding the k-th
+    // largest, then the few entries of Bt ranked pairwise (larger score
+    // first, lower index on ties; -0.0 == +0.0 as floats).
+    bool fast = false;
+    const float range = hi - lo;
+    const float scale = (range > 0.f && range < INFINITY) ? __fdiv_rn((float)kNB * 0.99999f, range) : 0.f;
+    if (scale > 0.f) {
+        for (int i = tid; i < total; i += kThreads)
+            atomicAdd(&sm.hist[bucket_of(__uint_as_float(sm.ckey[i]), lo, scale)], 1u);
+        __syncthreads();
+        find_threshold_bin(sm.hist, (uint32_t)k, sm.red, sm.bcast);
+        const uint32_t Bt = sm.bcast[0], need = sm.bcast[1];
+        const uint32_t in_bt = sm.hist[Bt];
+        __syncthreads();
+        if (in_bt <= (uint32_t)kMaxTies) {
+            fast = true;
+            uint32_t *tlist = sm.hist;  // [2 * kMaxTies]: (slot, index) of the entries in Bt
+            if (tid == 0) sm.bcast[3] = 0u;
+            __syncthreads();
+            for (int i = tid; i < total; i += kThreads) {
+                const uint32_t b = bucket_of(__uint_as_float(sm.ckey[i]), lo, scale);
+                if (!use_bits) sm.flag[i] = 0;
+                if (b > Bt) {
+                    mark(i);
+                } else if (b == Bt) {
+                    const uint32_t p = atomicAdd(&sm.bcast[3], 1u);
+                    tlist[2 * p] = (uint32_t)i;
+                    tlist[2 * p + 1] = (uint32_t)sm.cidx[i];
+                }
+            }
+            __syncthreads();
+            for (int i = tid; i < (int)in_bt; i += kThreads) {
+                const uint32_t si = tlist[2 * i];
+                const float vi = __uint_as_float(sm.ckey[si]);
+                const int32_t xi = (int32_t)tlist[2 * i + 1];
+                uint32_t before = 0;
+                for (int j2 = 0; j2 < (int)in_bt; ++j2) {
+                    const float vj = __uint_as_float(sm.ckey[tlist[2 * j2]]);
+                    before += vj > vi || (vj == vi && (int32_t)tlist[2 * j2 + 1] < xi);
+                }
+                if (before < need) mark((int)si);
+            }
+            __syncthreads();
+        }
+    }
+    if (!fast) {
+        // exact radix select over the 32-bit order keys (a row whose range
+        // is empty or whose threshold bucket is crowded)
+        for (int i = tid; i < total; i += kThreads) sm.ckey[i] = order_key(__uint_as_float(sm.ckey[i]));
+        __syncthreads();
+        // T = the k-th largest key; quota = how many entries equal to T are taken
+        uint32_t T, quota;
+        select_in_candidates(sm, total, (uint32_t)k, T, quota);
+        const uint32_t tied = sm.hist[T & 1023u];  // the last pass's bin of T holds every entry equal to T
+        __syncthreads();
+        if (tied > (uint32_t)kMaxTies) {
+            if (tid == 0) flag_repair(repair, r);
+            return;
+        }
+        // entries equal to T: the quota lowest indices (ranked pairwise in a
+        // short list kept in the histogram's space)
+        uint32_t *tlist = sm.hist;  // [2 * kMaxTies]: (slot, index)
         if (tid == 0) sm.bcast[3] = 0u;
         __syncthreads();
-        for (int i = tid; i < total; i += kThreads)
-            if (sm.ckey[i] == T) {
+        for (int i = tid; i < total; i += kThreads) {
+            if (!use_bits) sm.flag[i] = 0;
+            if (sm.ckey[i] > T) {
+                mark(i);
+            } else if (sm.ckey[i] == T) {
                 const uint32_t p = atomicAdd(&sm.bcast[3], 1u);
                 tlist[2 * p] = (uint32_t)i;
                 tlist[2 * p + 1] = (uint32_t)sm.cidx[i];
             }
+        }
         __syncthreads();
         for (int i = tid; i < (int)tied; i += kThreads) {
             const int32_t xi = (int32_t)tlist[2 * i + 1];
             uint32_t before = 0;
-            for (int j = 0; j < (int)tied; ++j) before += (int32_t)tlist[2 * j + 1] < xi;
-            // mark a tied entry that is not taken by clearing its key
-            if (before >= quota) sm.ckey[tlist[2 * i]] = 0u;
+            for (int j2 = 0; j2 < (int)tied; ++j2) before += (int32_t)tlist[2 * j2 + 1] < xi;
+            if (before < quota) mark((int)tlist[2 * i]);
         }
         __syncthreads();
     }
-    // selected: key > T, or key == T and still marked.  (A key of 0 is
-    // below every real score's key, so the cleared ties drop out.)
-    // Compact in slot order: each thread takes a run of consecutive slots.
+    if (use_bits) {
+        // the k set bits, in index order: each thread scans a run of words
+        const int per = (words + kThreads - 1) / kThreads;
+        const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
+        uint32_t mine = 0;
+        for (int w = w0; w < w1; ++w) mine += __popc(sm.bits[w]);
+        uint32_t tot;
+        uint32_t pos = block_scan_packed(mine, sm.red, &tot);
+        for (int w = w0; w < w1; ++w) {
+            uint32_t v = sm.bits[w];
+            while (v) {
+                const int b = __ffs(v) - 1;
+                v &= v - 1u;
+                out[pos++] = w * 32 + b;
+            }
+        }
+        return;
+    }
+    // Longer rows: compact the selected entries in slot order (each thread
+    // takes a run of consecutive slots), then merge the four ascending
+    // segment lists.
     const int per = (total + kThreads - 1) / kThreads;
     const int i0 = min(total, tid * per), i1 = min(total, i0 + per);
     uint32_t mine = 0;
-    for (int i = i0; i < i1; ++i) mine += sm.ckey[i] >= T && sm.ckey[i] != 0u;
+    for (int i = i0; i < i1; ++i) mine += sm.flag[i];
     uint32_t tot;
     uint32_t pos = block_scan_packed(mine, sm.red, &tot);
     // segment q's selected entries start at the rank of its first slot
@@ -239,17 +405,17 @@ __global__ void __launch_bounds__(kThreads) cand_select_kernel(const int2 *__res
         const int b = sm.seg_off[q];
         if (b >= i0 && b < i1) {
             uint32_t p = pos;
-            for (int i = i0; i < b; ++i) p += sm.ckey[i] >= T && sm.ckey[i] != 0u;
+            for (int i = i0; i < b; ++i) p += sm.flag[i];
             sm.sel_off[q] = (int)p;
         } else if (b == total && tid == 0) {
             sm.sel_off[q] = (int)tot;
         }
     }
     for (int i = i0; i < i1; ++i)
-        if (sm.ckey[i] >= T && sm.ckey[i] != 0u) sm.sel[pos++] = sm.cidx[i];
+        if (sm.flag[i]) sm.sel[pos++] = sm.cidx[i];
     __syncthreads();
-    // merge the four ascending lists: an entry's output position is its rank
-    // in its own list plus the entries of the other lists with a lower index
+    // an entry's output position is its rank in its own list plus the
+    // entries of the other lists with a lower index
     for (int p = tid; p < k; p += kThreads) {
         int q = 0;
         while (q < kSegs - 1 && p >= sm.sel_off[q + 1]) ++q;
