@@ -16,6 +16,8 @@ states the passage of the pages it follows:
   5.1.2 (rows below k keep all of [0, t]) and 5.2.1 (deterministic top-k).
 * attention -- same formula block, GQA sparse aggregation u_{t,g}; report
   section 2.3.2 (one index set for every group).
+* indexer_kl -- same formula block, the dense warm-up and sparse adaptation
+  losses of the indexer; report section 2.3.3.
 """
 from __future__ import annotations
 
@@ -68,8 +70,9 @@ def _load():
         lib.dsa_oracle_sparse_attention.argtypes = [P, P, P, P, I, I, I, I, I, I, D, P, P]
         lib.dsa_oracle_decode_indexer.argtypes = [P, P, P, P, P, P, I, I, I, P, I, I, I, P, I64]
         lib.dsa_oracle_decode_attention.argtypes = [P, P, P, P, I, I, I, P, P, I, I, I, I, I, D, P, P]
+        lib.dsa_oracle_indexer_kl.argtypes = [P, I64, I, I, P, I, I64, P, I, P, P]
         for f in ("dsa_oracle_indexer", "dsa_oracle_topk", "dsa_oracle_sparse_attention",
-                  "dsa_oracle_decode_indexer", "dsa_oracle_decode_attention"):
+                  "dsa_oracle_decode_indexer", "dsa_oracle_decode_attention", "dsa_oracle_indexer_kl"):
             getattr(lib, f).restype = I
         _lib = lib
     return _lib
@@ -214,6 +217,30 @@ def decode_attention(q, k_cache, v_cache, block_table, seq_lens, idx, sm_scale: 
                                                page, k_cache.shape[0], _p(seq_lens), _p(idx), B, Hq, Hkv, D, k,
                                                float(sm_scale), _p(out), _p(lse)), "decode_attention")
     return out, lse
+
+
+def indexer_kl(I, p, row_begin: int = 0, idx=None):
+    """Indexer distillation loss per query row ("Kwai Keye-VL-2.0 Technical
+    Report" review, 核心公式, dense warm-up / sparse adaptation losses;
+    report translation section 2.3.3):
+        sum_g KL( p[t,S,g] / sum_S p[t,S,g]  ||  Softmax(I[t,S]) )
+    with S = [0, t] (idx None: dense warm-up) or the valid entries of idx
+    row r (sparse adaptation).  I [n_rows, >= row_begin+n_rows] scores,
+    p [n_rows, G, >= row_begin+n_rows] non-negative target weights.
+    Returns (loss per row float64 [n_rows], total)."""
+    I = _c(I, np.float64)
+    p = _c(p, np.float64)
+    n_rows, ld_I = I.shape
+    _, G, ld_p = p.shape
+    k = 0
+    if idx is not None:
+        idx = _c(idx, np.int32)
+        k = idx.shape[1]
+    loss = np.empty(n_rows, np.float64)
+    total = np.empty(1, np.float64)
+    _check(_load().dsa_oracle_indexer_kl(_p(I), ld_I, row_begin, n_rows, _p(p), G, ld_p,
+                                         None if idx is None else _p(idx), k, _p(loss), _p(total)), "indexer_kl")
+    return loss, float(total[0])
 
 
 def prefill(q8, sq, w, k8, sk, Q, K, V, k: int, sm_scale: float, rows=None):

@@ -339,3 +339,73 @@ EXPORT int dsa_oracle_decode_attention(const uint16_t *q, const uint16_t *k_cach
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Indexer distillation losses                                         */
+/* ------------------------------------------------------------------ */
+
+/* [REVIEW] 核心公式, dense warm-up and sparse adaptation losses of the
+ * indexer; [REPORT] 2.3.3 (the target of group g is the group's aggregated
+ * dense attention, normalised; in the sparse stage it is truncated to the
+ * selected set S_t and renormalised, and the softmax of the indexer scores is
+ * taken over S_t only):
+ *   dense:  L = sum_t sum_g KL( p[t,:,g]   || Softmax(I[t,:])   )
+ *   sparse: L = sum_t sum_g KL( p[t,S_t,g] || Softmax(I[t,S_t]) )
+ * KL(a || b) = sum_s a_s log(a_s / b_s), with 0 log 0 = 0.
+ *
+ * Row r is query t = row_begin + r.  I [n_rows, ld_I]: scores of keys
+ * 0..t.  p [n_rows, G, ld_p]: non-negative target weights of keys 0..t
+ * (normalised here over the set, so a scaled target gives the same loss).
+ * idx NULL: S_t = [0, t] (dense); otherwise S_t = the entries of idx row r
+ * that lie in [0, t] (k of them at most, -1 padded, distinct).
+ * Readings: the causal range [0, t] is the one the indexer scores; a group
+ * whose target has no mass on S_t contributes 0.
+ * loss [n_rows] receives sum_g KL for each row, *total their sum. */
+EXPORT int dsa_oracle_indexer_kl(const double *I, int64_t ld_I, int row_begin, int n_rows,
+                                 const double *p, int G, int64_t ld_p, const int32_t *idx, int k,
+                                 double *loss, double *total)
+{
+    if (row_begin < 0 || n_rows < 0 || G < 1 || (idx && k < 1)) return -1;
+    if (ld_I < row_begin + n_rows || ld_p < row_begin + n_rows) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < n_rows; ++r) {
+        int t = row_begin + r;
+        /* the set S_t */
+        int n = idx ? 0 : t + 1;
+        int32_t *S = (int32_t *)malloc(sizeof(int32_t) * (size_t)(idx ? k : t + 1));
+        if (idx) {
+            for (int i = 0; i < k; ++i) {
+                int32_t s = idx[(size_t)r * k + i];
+                if (s >= 0 && s <= t) S[n++] = s;
+            }
+        } else {
+            for (int s = 0; s <= t; ++s) S[s] = s;
+        }
+        const double *Ir = I + (size_t)r * ld_I;
+        /* Softmax(I[t, S]) as log-probabilities: log q_s = I_s - log sum_u exp(I_u) */
+        double mx = -INFINITY;
+        for (int i = 0; i < n; ++i) if (Ir[S[i]] > mx) mx = Ir[S[i]];
+        double z = 0.0;
+        for (int i = 0; i < n; ++i) z += exp(Ir[S[i]] - mx);
+        double logz = mx + log(z);
+        double row_loss = 0.0;
+        for (int g = 0; g < G; ++g) {
+            const double *pr = p + ((size_t)r * G + g) * ld_p;
+            double mass = 0.0;
+            for (int i = 0; i < n; ++i) mass += pr[S[i]];
+            if (!(mass > 0.0)) continue;
+            double kl = 0.0;
+            for (int i = 0; i < n; ++i) {
+                double a = pr[S[i]] / mass;
+                if (a > 0.0) kl += a * (log(a) - (Ir[S[i]] - logz));
+            }
+            row_loss += kl;
+        }
+        loss[r] = row_loss;
+        free(S);
+    }
+    double sum = 0.0;
+    for (int r = 0; r < n_rows; ++r) sum += loss[r];
+    *total = sum;
+    return 0;
+}

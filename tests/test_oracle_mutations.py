@@ -4,7 +4,8 @@ Each case copies the oracle's C source, plants one mistake of the kind a
 reader could make when writing the formulas of "Kwai Keye-VL-2.0 Technical
 Report" review (xllm-io), 核心公式, and report translation sections 2.3.1 /
 2.3.2 (a dropped ReLU or scale, a wrong sign or index, a reversed tie rule, a
-wrong GQA group map, a missing normalisation, a wrong FP8 exponent bias),
+wrong GQA group map, a missing normalisation, a wrong FP8 exponent bias) and
+2.3.3 (the indexer's distillation losses),
 compiles it with gcc, and runs the pin suite against that copy in a fresh
 process.  The pin suite must fail for every one of them.  Everything runs on
 the CPU.
@@ -34,6 +35,11 @@ MUTATIONS = {
     "sm_scale_dropped": ("logit[i] = sm_scale * dot;", "logit[i] = dot;"),
     "e4m3_bias_off": ("mag = ldexp(1.0 + (double)m / 8.0, e - 7);", "mag = ldexp(1.0 + (double)m / 8.0, e - 8);"),
     "e4m3_subnormal_scale": ("mag = ldexp((double)m / 8.0, 1 - 7);", "mag = ldexp((double)m / 8.0, -7);"),
+    "kl_sign_flipped": ("if (a > 0.0) kl += a * (log(a) - (Ir[S[i]] - logz));",
+                        "if (a > 0.0) kl += a * ((Ir[S[i]] - logz) - log(a));"),
+    "kl_target_not_renormalised": ("double a = pr[S[i]] / mass;", "double a = pr[S[i]];"),
+    "kl_softmax_not_normalised": ("double logz = mx + log(z);", "double logz = mx;"),
+    "kl_sparse_padding_counted": ("if (s >= 0 && s <= t) S[n++] = s;", "if (s <= t) S[n++] = s < 0 ? 0 : s;"),
     "page_slot_swapped": ("size_t slot = (size_t)p * page + (size_t)(s % page);\n            out[(size_t)b * ld + s]",
                           "size_t slot = (size_t)p * page + (size_t)((page - 1) - s % page);\n            out[(size_t)b * ld + s]"),
 }

@@ -407,3 +407,116 @@ def test_oracle_results_do_not_depend_on_thread_count(oracle_mod):
     finally:
         oracle_mod.set_threads(n0)
     assert np.array_equal(a, b)
+
+
+# ----------------------------------------------------------------------------
+# indexer distillation losses (dense warm-up, sparse adaptation)
+# ----------------------------------------------------------------------------
+
+def test_indexer_kl_hand_example(oracle_mod):
+    g = read_golden("indexer_kl_hand_example.txt")
+    I = np.array([g["dense_I"]])                      # row t = 1
+    p = np.array([[g["dense_p_g0"], g["dense_p_g1"]]])
+    loss, total = oracle_mod.indexer_kl(I, p, row_begin=1)
+    assert loss[0] == pytest.approx(g["dense_loss"][0], rel=1e-14)
+    assert total == pytest.approx(g["dense_loss"][0], rel=1e-14)
+    I = np.array([g["sparse_I"]])                     # row t = 2
+    p = np.array([[g["sparse_p"]]])
+    idx = np.array([[int(x) for x in g["sparse_idx"]]], np.int32)
+    loss, _ = oracle_mod.indexer_kl(I, p, row_begin=2, idx=idx)
+    assert loss[0] == pytest.approx(g["sparse_loss"][0], rel=1e-14)
+
+
+def _kl_case(seed, n_rows=6, L=40, G=3, zeros=True):
+    rng = np.random.default_rng(seed)
+    I = rng.normal(0, 3, (n_rows, L))
+    p = rng.random((n_rows, G, L)) ** 3
+    if zeros:
+        p[rng.random(p.shape) < 0.3] = 0.0
+    return I, p
+
+
+def test_indexer_kl_matches_scipy_entropy(oracle_mod):
+    # scipy.stats.entropy(pk, qk) normalises pk and qk and returns KL(pk || qk)
+    from scipy.special import softmax
+    from scipy.stats import entropy
+    I, p = _kl_case(1)
+    r0 = 30
+    loss, total = oracle_mod.indexer_kl(I, p, row_begin=r0)
+    for r in range(I.shape[0]):
+        t = r0 + r
+        q = softmax(I[r, : t + 1])
+        ref = sum(entropy(p[r, g, : t + 1], q) for g in range(p.shape[1]))
+        assert loss[r] == pytest.approx(ref, rel=1e-12, abs=1e-14)
+    assert total == pytest.approx(loss.sum(), rel=1e-14)
+
+
+def test_indexer_kl_zero_when_target_is_the_indexer_softmax(oracle_mod):
+    from scipy.special import softmax
+    rng = np.random.default_rng(2)
+    L, r0 = 20, 14
+    I = rng.normal(0, 2, (6, L))
+    p = np.zeros((6, 2, L))
+    for r in range(6):
+        t = r0 + r
+        for g, c in enumerate((1.0, 7.5)):   # any positive multiple of the softmax
+            p[r, g, : t + 1] = softmax(I[r, : t + 1]) * c
+    loss, _ = oracle_mod.indexer_kl(I, p, row_begin=r0)
+    assert np.all(np.abs(loss) < 1e-12)
+
+
+def test_indexer_kl_invariances_and_sign(oracle_mod):
+    I, p = _kl_case(3)
+    r0 = 34
+    base, _ = oracle_mod.indexer_kl(I, p, row_begin=r0)
+    assert np.all(base > 0)                                        # Gibbs: KL >= 0
+    shifted, _ = oracle_mod.indexer_kl(I + 11.25, p, row_begin=r0)  # softmax is shift invariant
+    np.testing.assert_allclose(shifted, base, rtol=1e-11)
+    scaled, _ = oracle_mod.indexer_kl(I, p * 3.5, row_begin=r0)     # the target is normalised
+    np.testing.assert_allclose(scaled, base, rtol=1e-12)
+    # entries right of the causal range take no part
+    I2, p2 = I.copy(), p.copy()
+    for r in range(I.shape[0]):
+        I2[r, r0 + r + 1:] = 1e3
+        p2[r, :, r0 + r + 1:] = 5.0
+    np.testing.assert_allclose(oracle_mod.indexer_kl(I2, p2, row_begin=r0)[0], base, rtol=1e-14)
+
+
+def test_indexer_kl_sparse_over_every_causal_key_is_dense(oracle_mod):
+    I, p = _kl_case(4)
+    r0 = 34
+    dense, _ = oracle_mod.indexer_kl(I, p, row_begin=r0)
+    k = 48
+    rng = np.random.default_rng(5)
+    idx = np.full((I.shape[0], k), -1, np.int32)
+    for r in range(I.shape[0]):
+        idx[r, : r0 + r + 1] = rng.permutation(r0 + r + 1)
+    sparse, _ = oracle_mod.indexer_kl(I, p, row_begin=r0, idx=idx)
+    np.testing.assert_allclose(sparse, dense, rtol=1e-12)
+
+
+def test_indexer_kl_sparse_is_dense_on_the_truncated_row(oracle_mod):
+    # the sparse loss over S equals the dense loss of a row that holds only
+    # the keys of S (the target renormalised over S, the softmax over S)
+    from scipy.special import softmax
+    from scipy.stats import entropy
+    I, p = _kl_case(6, n_rows=4, L=40, G=2)
+    r0 = 36
+    rng = np.random.default_rng(7)
+    idx = np.full((4, 9), -1, np.int32)
+    for r in range(4):
+        idx[r, :7] = rng.choice(r0 + r + 1, 7, replace=False)
+    sparse, _ = oracle_mod.indexer_kl(I, p, row_begin=r0, idx=idx)
+    for r in range(4):
+        S = idx[r, :7]
+        ref = sum(entropy(p[r, g, S], softmax(I[r, S])) if p[r, g, S].sum() > 0 else 0.0 for g in range(2))
+        assert sparse[r] == pytest.approx(ref, rel=1e-12, abs=1e-14)
+
+
+def test_indexer_kl_group_without_mass_contributes_nothing(oracle_mod):
+    I, p = _kl_case(8, n_rows=3, L=12, G=2, zeros=False)
+    r0 = 9
+    base, _ = oracle_mod.indexer_kl(I, p[:, :1], row_begin=r0)
+    p[:, 1] = 0.0
+    both, _ = oracle_mod.indexer_kl(I, p, row_begin=r0)
+    np.testing.assert_allclose(both, base, rtol=1e-15)
