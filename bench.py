@@ -98,10 +98,10 @@ def measure_read_peaks(dsa):
     stream = torch.cuda.current_stream()
     sink = torch.zeros(4, dtype=torch.int32, device="cuda")
     l2 = {}
-    for mb in (16, 32, 48, 64):
+    for mb in (8, 16, 24, 32, 48, 64):
         buf = torch.ones(mb << 18, dtype=torch.int32, device="cuda")
-        reps = 64
-        ms = _best_ms(lambda: dsa.read_probe(buf, reps, sink), 5, stream)
+        reps = max(64, 2048 // mb)
+        ms = _best_ms(lambda: dsa.read_probe(buf, reps, sink), 10, stream)
         l2[mb] = reps * buf.numel() * 4 / (ms / 1e3) / 1e9
         del buf
     big = torch.ones(1 << 30, dtype=torch.int32, device="cuda")
@@ -110,7 +110,7 @@ def measure_read_peaks(dsa):
     del big
     best_mb = max(l2, key=l2.get)
     return {"l2_read_gbs": l2[best_mb], "l2_read_gbs_by_mb": l2, "hbm_read_gbs": hbm_read,
-            "how": f"dsa_read_probe: {best_mb} MiB buffer read 64 times (best of 16/32/48/64 MiB, best of 5); "
+            "how": f"dsa_read_probe: {best_mb} MiB buffer read repeatedly (best of 8-64 MiB buffers, best of 10); "
                    f"HBM: one pass over 4 GiB, best of 5; CUDA events"}
 
 
@@ -430,6 +430,37 @@ def run_prefill_e2e(pb, steps, warmup):
     return ms, h2d_bytes, d2h_bytes
 
 
+def run_kl_timed(dsa, inputs, pk, reps=5, n_rows=4096, G=4):
+    """The indexer's distillation losses (dense warm-up over every causal key,
+    sparse adaptation over Omega_t) on the last n_rows query rows of the
+    32K layer, against HBM: algorithmic bytes are the scores and G target
+    weights of every key visited (plus the index rows for the sparse loss)."""
+    cfg = inputs.config(1)
+    d = inputs.prefill_inputs(cfg, device="cuda")
+    L, k = cfg.L, cfg.k
+    r0 = L - n_rows
+    scores = torch.empty(n_rows, L, dtype=torch.float32, device="cuda")
+    dsa.indexer_scores(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], r0, n_rows, scores)
+    need = dsa.topk_workspace_size(n_rows, L, k)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda") if need else None
+    idx = torch.empty(n_rows, k, dtype=torch.int32, device="cuda")
+    dsa.topk(scores, r0, n_rows, k, idx, max_len=L, ws=ws)
+    del d
+    p = inputs.kl_targets(n_rows, G, L, seed=77, device="cuda")
+    loss = torch.empty(n_rows, dtype=torch.float64, device="cuda")
+    total = torch.empty(1, dtype=torch.float64, device="cuda")
+    stream = torch.cuda.current_stream()
+    out = {"workload": f"prefill-32k rows {r0}..{L - 1} ({n_rows} rows), G={G} target groups, k={k}"}
+    keys = sum(t + 1 for t in range(r0, L))
+    for name, ix, byts in (("dense", None, keys * (4 + 4 * G)), ("sparse", idx, n_rows * k * (4 + 4 + 4 * G))):
+        ms = _best_ms(lambda: dsa.indexer_kl(scores, r0, n_rows, p, loss, idx=ix, loss_total=total), reps, stream)
+        gbs = byts / (ms / 1e3) / 1e9
+        out[name] = {"ms": ms, "bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / pk["hbm_gbs"], "algorithmic_bytes": byts}
+    dsa.check_device_error()
+    return out
+
+
 class DecodeBench:
     def __init__(self, cfg, seed, device, batch=None):
         from sparse_long_context_03_b200 import dsa, inputs
@@ -713,6 +744,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--chunk-rows", type=int, default=None,
                     help="query rows per indexer/top-k chunk (default: a 4 GiB score block)")
+    ap.add_argument("--no-kl", action="store_true", help="skip the indexer distillation-loss leg")
     ap.add_argument("--unfused", action="store_true",
                     help="materialise the score matrix per chunk and run dsa_topk (instead of dsa_indexer_topk)")
     ap.add_argument("--decode-batch", type=int, default=None,
@@ -789,6 +821,12 @@ def main():
         torch.cuda.empty_cache()
         pb = None
 
+    kl = None
+    if rank == 0 and not args.no_kl:
+        from sparse_long_context_03_b200 import dsa as _dsa_kl
+        kl = run_kl_timed(_dsa_kl, inputs, pk)
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         d_cpu = inputs.prefill_inputs(cfg, device="cuda", seed=cfg.seed)
@@ -810,7 +848,7 @@ def main():
                              "candidate lists or 4 GiB score chunks)"},
             "roofline": dom_line, "stages": stages, "clocks": clocks, "gpu_launches": None,
             "peaks_measured_here": {"fp8": fp8, "reads": reads},
-            "e2e": e2e, "decode": decode, "cpu_baseline": cpu,
+            "e2e": e2e, "decode": decode, "indexer_kl": kl, "cpu_baseline": cpu,
         }
         # kernels per library call: the fused threshold stage runs the sampled indexer and the threshold
         # select, the select stage the candidate select, the repair kernel and the stats copy

@@ -72,6 +72,14 @@ DSA_API const char *dsa_last_error_string(void);
  * expired since the last call (the kernel then wrote incomplete results and
  * exited cleanly), DSA_OK otherwise.  Clears the flag. */
 DSA_API dsa_status_t dsa_check_device_error(void);
+/* Diagnostic, for tests of the failure path: sets, on the current device,
+ * the time after which the prefill indexer's on-chip pipeline waits (between
+ * its TMA, tensor-core and epilogue roles) give up, in nanoseconds; 0
+ * restores the default of 2 s.  A wait that gives up sets the flag that
+ * dsa_check_device_error reports, every role of the kernel unwinds (copies in
+ * flight are drained, tensor memory is freed) and the scores are incomplete.
+ * Synchronous; not for the hot path. */
+DSA_API dsa_status_t dsa_set_wait_limit_ns(unsigned long long ns);
 
 /* ------------------------------------------------------------------------
  * Lightning-indexer scores (prefill), one chunk of query rows.
@@ -191,6 +199,34 @@ DSA_API dsa_status_t dsa_indexer_topk_select(const uint8_t *q8, const float *q_s
                               int32_t *idx, void *ws, size_t ws_bytes, int64_t *stats, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Indexer distillation losses (forward), one chunk of query rows.
+ *
+ * [REVIEW] 核心公式, dense warm-up loss and sparse adaptation loss;
+ * [REPORT] 2.3.3 (the target of group g is its aggregated dense attention,
+ * normalised; in the sparse stage it is truncated to the selected set S_t and
+ * renormalised, and the indexer softmax runs over S_t):
+ *     loss_rows[r] = sum_{g<G} KL( p[r,g,S] / sum_S p[r,g,S]  ||  Softmax(I[t,S]) )
+ *     KL(a||b) = sum_s a_s ln(a_s / b_s),  0 ln 0 = 0,   t = row_begin + r.
+ *   idx == NULL: S = [0, t] (dense warm-up); otherwise S = the entries of idx
+ *   row r that lie in [0, t] (sparse adaptation; entries must be distinct,
+ *   -1 padding and out-of-range entries are skipped).
+ *
+ *   scores     [n_rows, ld_scores] float: I[t, s] for s <= t (e.g. from
+ *              dsa_indexer_scores); ld_scores >= row_begin + n_rows.
+ *   p          [n_rows, G, ld_p] float, non-negative target weights for keys
+ *              0..t (they are normalised over S here); ld_p >= row_begin + n_rows.
+ *   idx        NULL, or [n_rows, k] int32 (e.g. from dsa_topk).
+ *   loss_rows  [n_rows] double: the loss of each row; a group with no target
+ *              mass on S contributes 0, a row whose S is empty gets 0.
+ *   loss_total optional (NULL to skip): one double, the sum of loss_rows
+ *              (fixed summation order: bitwise reproducible).
+ * Sums are accumulated in double precision from the float inputs.
+ * ------------------------------------------------------------------------ */
+DSA_API dsa_status_t dsa_indexer_kl(const float *scores, int64_t ld_scores, int row_begin, int n_rows,
+                            const float *p, int G, int64_t ld_p, const int32_t *idx, int k,
+                            double *loss_rows, double *loss_total, void *stream);
+
+/* ------------------------------------------------------------------------
  * Sparse GQA attention (prefill), one chunk of query rows.
  *
  * [REVIEW] 核心公式, u[t,g] = Attn(h[t,g], { c[s,g] | s in Omega_t });
@@ -292,6 +328,9 @@ DSA_API dsa_status_t dsa_sparse_gqa_decode_attention(const uint16_t *q,
  *    workspace variant's, so results can differ from it by rounding only.
  *  - The first call on a device looks up the array's device address with
  *    that device current; make that first call before any stream capture.
+ *    The address is kept for the life of the process: after a
+ *    cudaDeviceReset of that device it is stale, so do not call this entry
+ *    point on a device that has been reset.
  *  - Every call on a device shares the one array: calls whose executions
  *    overlap on the GPU (other streams, other host threads) race.  Nothing
  *    has to be cleared between calls; each call writes every partial it reads.

@@ -79,6 +79,8 @@ dsa_status_t dsa_check_device_error(void) {
     return flag ? DSA_ERR_TIMEOUT : DSA_OK;
 }
 
+dsa_status_t dsa_set_wait_limit_ns(unsigned long long ns) { return cuda_status(dsa::indexer_tc_set_wait_limit(ns)); }
+
 size_t dsa_row_stats_bytes(int n_rows) { return n_rows > 0 ? (size_t)n_rows * 8 * sizeof(float) : 0; }
 
 dsa_status_t dsa_indexer_scores(const uint8_t *q8, const float *q_scale, const float *w, const uint8_t *k8,
@@ -189,6 +191,18 @@ dsa_status_t dsa_indexer_topk_select(const uint8_t *q8, const float *q_scale, co
     const Range range(__func__);
     return indexer_topk_checked(3, q8, q_scale, w, k8, k_scale, L, HI, dI, row_begin, n_rows, k, idx, ws, ws_bytes,
                                 stats, stream);
+}
+
+dsa_status_t dsa_indexer_kl(const float *scores, int64_t ld_scores, int row_begin, int n_rows, const float *p,
+                            int G, int64_t ld_p, const int32_t *idx, int k, double *loss_rows, double *loss_total,
+                            void *stream) {
+    const Range range(__func__);
+    if (row_begin < 0 || n_rows < 0 || G < 1 || (idx != nullptr && k < 1)) return DSA_ERR_INVALID_ARG;
+    if (n_rows == 0 && loss_total == nullptr) return DSA_OK;
+    if ((n_rows > 0 && (!scores || !p || !loss_rows)) || (n_rows == 0 && !loss_rows)) return DSA_ERR_INVALID_ARG;
+    if (ld_scores < (int64_t)row_begin + n_rows || ld_p < (int64_t)row_begin + n_rows) return DSA_ERR_INVALID_ARG;
+    return cuda_status(dsa::launch_indexer_kl(scores, ld_scores, row_begin, n_rows, p, G, ld_p, idx,
+                                              idx ? k : 0, loss_rows, loss_total, as_stream(stream)));
 }
 
 dsa_status_t dsa_sparse_gqa_prefill(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const int32_t *idx,

@@ -25,6 +25,8 @@ cudaError_t launch_indexer_prefill_tc(const uint8_t *q8, const float *sq, const 
                                       const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
                                       float *scores, int64_t ld, float *row_stats, cudaStream_t stream);
 cudaError_t indexer_tc_take_error(unsigned int *flag);
+// bound of the prefill indexer's pipeline waits on the current device (0: the default)
+cudaError_t indexer_tc_set_wait_limit(unsigned long long ns);
 // the same kernel scoring every indexer_sample_stride()-th key only:
 // sample_scores [n_rows, ld], column j = key j * stride (causal: j * stride <= t)
 int indexer_sample_stride();
@@ -68,6 +70,11 @@ cudaError_t launch_indexer_topk_stage(int stage, const uint8_t *q8, const float 
                                       const uint8_t *k8, const float *sk, int L, int HI, int dI, int row_begin,
                                       int n_rows, int k, int32_t *idx, void *ws, int64_t *stats,
                                       cudaStream_t stream);
+
+// indexer_kl.cu: the indexer's distillation losses (forward)
+cudaError_t launch_indexer_kl(const float *scores, int64_t ld, int row_begin, int n_rows, const float *p, int G,
+                              int64_t ld_p, const int32_t *idx, int k, double *loss_rows, double *loss_total,
+                              cudaStream_t stream);
 
 // attention.cu
 bool attention_shape_supported(int Hq, int Hkv, int D);

@@ -33,6 +33,7 @@ _SIGNATURES = {
     "dsa_version": ([], _I),
     "dsa_last_error_string": ([], ctypes.c_char_p),
     "dsa_check_device_error": ([], _I),
+    "dsa_set_wait_limit_ns": ([ctypes.c_ulonglong], _I),
     "dsa_row_stats_bytes": ([_I], _SZ),
     "dsa_indexer_scores": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P, _P], _I),
     "dsa_topk_workspace_size": ([_I, _I, _I], _SZ),
@@ -42,6 +43,7 @@ _SIGNATURES = {
     "dsa_indexer_topk_threshold": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P, _P], _I),
     "dsa_indexer_topk_candidates": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P, _P], _I),
     "dsa_indexer_topk_select": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P, _P], _I),
+    "dsa_indexer_kl": ([_P, _I64, _I, _I, _P, _I, _I64, _P, _I, _P, _P, _P], _I),
     "dsa_sparse_gqa_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P], _I),
     "dsa_decode_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
     "dsa_sparse_gqa_decode": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _I,
@@ -87,6 +89,17 @@ def status_string(code: int) -> str:
 def check_device_error():
     """Synchronises; raises DSAError if a kernel's bounded wait expired."""
     _check(lib().dsa_check_device_error(), "dsa_check_device_error")
+
+
+def device_error_status() -> int:
+    """dsa_check_device_error's status code (0 = none), without raising."""
+    return int(lib().dsa_check_device_error())
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """dsa_set_wait_limit_ns: bound of the prefill indexer's pipeline waits
+    on the current device (0 restores the default).  For failure-path tests."""
+    _check(lib().dsa_set_wait_limit_ns(int(ns)), "dsa_set_wait_limit_ns")
 
 
 def _check(code: int, name: str):
@@ -189,6 +202,24 @@ def indexer_topk(q8, q_scale, w, k8, k_scale, row_begin, n_rows, k, idx, ws, sta
     _check(getattr(lib(), name)(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), L, HI, dI,
                                 int(row_begin), int(n_rows), int(k), _ptr(idx), _ptr(ws),
                                 ws.numel() * ws.element_size(), _ptr(stats), _stream(stream)), name)
+
+
+def indexer_kl(scores, row_begin, n_rows, p, loss_rows, idx=None, loss_total=None, stream=None):
+    """dsa_indexer_kl: per-row indexer distillation loss
+    sum_g KL(p[r,g,S] normalised || Softmax(I[t,S])) into loss_rows [n_rows]
+    float64; S = [0, t] (idx None: dense warm-up) or the valid entries of idx
+    row r (sparse adaptation).  scores [n_rows, ld] float32, p [n_rows, G,
+    ld_p] float32; loss_total (optional, 1 float64) gets the sum."""
+    _need(scores, torch.float32, 2, "scores")
+    _need(p, torch.float32, 3, "p")
+    _need(loss_rows, torch.float64, 1, "loss_rows")
+    k = 0
+    if idx is not None:
+        _need(idx, torch.int32, 2, "idx")
+        k = idx.shape[1]
+    _check(lib().dsa_indexer_kl(_ptr(scores), scores.stride(0), int(row_begin), int(n_rows), _ptr(p), p.shape[1],
+                                p.stride(1), _ptr(idx), k, _ptr(loss_rows), _ptr(loss_total), _stream(stream)),
+           "dsa_indexer_kl")
 
 
 def sparse_gqa_prefill(Q, K, V, idx, row_begin, n_rows, k, sm_scale, O, lse=None, stream=None):

@@ -180,6 +180,16 @@ def exact_indexer_inputs(L: int, HI: int, dI: int, seed: int, device="cpu",
     return dict(q8=q8.contiguous(), sq=sq, w=w.contiguous(), k8=k8.contiguous(), sk=sk)
 
 
+def kl_targets(n_rows: int, G: int, width: int, seed: int, device="cpu", zero_frac: float = 0.3) -> torch.Tensor:
+    """Non-negative target weights [n_rows, G, width] float32 for the
+    indexer's distillation losses: U(0,1)^3 draws with a fraction of exact
+    zeros (the loss normalises them; nothing here is normalised)."""
+    g = _gen(device, seed)
+    x = torch.rand(n_rows, G, width, generator=g, device=device) ** 3
+    z = torch.rand(n_rows, G, width, generator=g, device=device) < zero_frac
+    return torch.where(z, torch.zeros_like(x), x).contiguous()
+
+
 def tie_heavy_scores(n_rows: int, width: int, seed: int, device="cpu") -> torch.Tensor:
     """fp32 score rows for exercising the top-k alone: a mix of clustered
     duplicates, signed zeros, negatives and a few large values."""
