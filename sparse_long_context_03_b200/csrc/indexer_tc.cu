@@ -41,6 +41,12 @@
 namespace dsa {
 
 __device__ unsigned int g_indexer_tc_error;
+// Bound of the prefill indexer's pipeline waits (between its TMA, MMA and
+// epilogue roles), in ns.  The default is far above any legitimate wait; a
+// test lowers it to make the waits give up and exercise the unwinding.  The
+// waits that drain copies in flight and the final MMA completion keep their
+// own fixed bounds.
+__device__ unsigned long long g_wait_limit_ns = 2000000000ull;
 
 namespace {
 
@@ -180,6 +186,7 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
     const int warp = threadIdx.x >> 5, lane = lane_id();
     const int row_end = row_begin + n_rows;
     const int nb = (n_rows + NQ - 1) / NQ;
+    const uint64_t wait_ns = g_wait_limit_ns;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -223,7 +230,7 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                 const int t_hi = min(t0 + NQ, row_end) - 1;
                 const int nstep = (t_hi / KS) / kStepKeys + 1;
                 const int qs = bi & 1;
-                if (!tc::mbar_wait_sleep(qempty_bar(qs), ((bi >> 1) & 1) ^ 1, kWaitLimitNs, kIssuerSleepNs)) {
+                if (!tc::mbar_wait_sleep(qempty_bar(qs), ((bi >> 1) & 1) ^ 1, wait_ns, kIssuerSleepNs)) {
                     ok = false;
                     break;
                 }
@@ -231,7 +238,7 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                 tc::tma_load_2d(sbase + Lay::kQ + qs * Lay::kQBytes, &tmap_q, 0, t0 * HI, qfull_bar(qs));
                 ++q_issued;
                 for (int st = 0; st < nstep; ++st) {
-                    if (!tc::mbar_wait_sleep(empty_bar(stage), phase ^ 1, kWaitLimitNs, kIssuerSleepNs)) {
+                    if (!tc::mbar_wait_sleep(empty_bar(stage), phase ^ 1, wait_ns, kIssuerSleepNs)) {
                         ok = false;
                         break;
                     }
@@ -267,7 +274,7 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                 const int t_hi = min(t0 + NQ, row_end) - 1;
                 const int nstep = (t_hi / KS) / kStepKeys + 1;
                 const int qs = bi & 1;
-                if (!tc::mbar_wait_sleep(qfull_bar(qs), (bi >> 1) & 1, kWaitLimitNs, kIssuerSleepNs)) {
+                if (!tc::mbar_wait_sleep(qfull_bar(qs), (bi >> 1) & 1, wait_ns, kIssuerSleepNs)) {
                     ok = false;
                     break;
                 }
@@ -277,9 +284,9 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                     if ((it & 1) != mw) continue;
                     const int pr = mw;
                     const int stage = it % kStages;
-                    if (!tc::mbar_wait_sleep(tempty_bar(pr), ((it / kPairs) & 1) ^ 1, kWaitLimitNs,
+                    if (!tc::mbar_wait_sleep(tempty_bar(pr), ((it / kPairs) & 1) ^ 1, wait_ns,
                                              kIssuerSleepNs) ||
-                        !tc::mbar_wait_sleep(full_bar(stage), (it / kStages) & 1, kWaitLimitNs, kIssuerSleepNs)) {
+                        !tc::mbar_wait_sleep(full_bar(stage), (it / kStages) & 1, wait_ns, kIssuerSleepNs)) {
                         ok = false;
                         break;
                     }
@@ -349,7 +356,7 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
             }
             for (int st = 0; st < nstep; ++st, ++it) {
                 const int pr = it % kPairs;
-                if (!tc::mbar_wait(tfull_bar(pr), (it / kPairs) & 1, kWaitLimitNs)) { ok = false; break; }
+                if (!tc::mbar_wait(tfull_bar(pr), (it / kPairs) & 1, wait_ns)) { ok = false; break; }
                 tc::tc_fence_after();
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
@@ -1009,6 +1016,11 @@ cudaError_t launch_indexer_cand_tc(const uint8_t *q8, const float *sq, const flo
 }
 
 int indexer_sample_stride() { return kSampleStride; }
+
+cudaError_t indexer_tc_set_wait_limit(unsigned long long ns) {
+    const unsigned long long v = ns ? ns : kWaitLimitNs;
+    return cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof v);
+}
 
 cudaError_t indexer_tc_take_error(unsigned int *flag) {
     unsigned int zero = 0;

@@ -90,3 +90,21 @@ def test_no_alloc_rejects_batches_beyond_its_scratch():
                                                      0.1, bogus, None, None)
     assert rc == 3  # DSA_ERR_WORKSPACE
     assert b"fixed decode scratch" in lib.dsa_last_error_string()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg_id,B", [(3, 504), (0, 1985)])
+def test_no_alloc_largest_accepted_batch(cfg_id, B):
+    # the largest batch whose partials fit the fixed array (B * Hkv * 8 *
+    # (D + 2) * 4 bytes <= 8 MiB): one split per (sequence, group), the
+    # partials reaching the end of the array
+    cfg = inputs.config(cfg_id)
+    assert B * cfg.Hkv * 8 * (cfg.D + 2) * 4 <= dsa.decode_attention_fixed_scratch_bytes()
+    assert (B + 1) * cfg.Hkv * 8 * (cfg.D + 2) * 4 > dsa.decode_attention_fixed_scratch_bytes()
+    rng = np.random.default_rng(B)
+    lens = [int(x) for x in rng.integers(1, 400, B)]
+    k = cfg.k
+    cfg, g, idx = _decode_case(cfg_id, lens, k, seed=80 + cfg_id)
+    _compare(_no_alloc(cfg, g, idx, k), _with_workspace(cfg, g, idx, k))
+    _compare(_no_alloc(cfg, g, idx, k), _with_workspace(cfg, g, idx, k))
+    torch.cuda.synchronize()
