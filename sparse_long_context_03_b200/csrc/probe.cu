@@ -5,7 +5,7 @@
 // DSA layer.
 //
 // Loads are 16-byte ld.global.cg (cached in L2 only, not in L1), the access
-// pattern of the attention's cp.async.cg gathers, four in flight per thread.
+// pattern of the attention's cp.async.cg gathers, eight in flight per thread.
 #include "kernels.h"
 
 namespace dsa {
@@ -21,7 +21,7 @@ __device__ __forceinline__ uint4 ld_cg_16(const uint4 *p) {
 }
 
 constexpr int kProbeThreads = 512;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 8;
 
 __global__ void __launch_bounds__(kProbeThreads) read_probe_kernel(const uint4 *__restrict__ buf, size_t n16, int reps,
                                                                   uint32_t *__restrict__ sink) {
