@@ -112,28 +112,6 @@ enum IndexerMode : int {
     kModeCand = 2,     // keep only scores >= the row's threshold, as (index, score) pairs
 };
 
-// ReLU on the FMA pipe: mul.sat clamps to [0, 1], so with d scaled by 2^-26
-// it returns d * 2^-26 for d >= 0 and 0 otherwise (|d| <= dI * 448^2 < 2^26
-// for e4m3 dot products up to dI = 128; the scaling by a power of two is
-// exact).  The head weight is pre-scaled by 2^26, so w' * y is exactly
-// w * ReLU(d) and the fused multiply-add rounds the same value as the fmax
-// path.  Five head pairs in eight take fmax (ALU pipe), three take mul.sat
-// (FMA pipe), which balances the two pipes against the issue rate.
-constexpr float kSatDown = 1.0f / 67108864.0f;  // 2^-26
-constexpr float kSatUp = 67108864.0f;           // 2^26
-#ifndef DSA_FMAX8
-constexpr int kFmaxPairsPer8 = 5;
-#else
-constexpr int kFmaxPairsPer8 = DSA_FMAX8;  // tuning builds only
-#endif
-__host__ __device__ constexpr bool sat_pair(int p) { return (p & 7) >= kFmaxPairsPer8; }
-
-__device__ __forceinline__ float relu_sat(float d) {
-    float y;
-    asm("mul.rn.sat.f32 %0, %1, %2;\n" : "=f"(y) : "f"(d), "f"(kSatDown));
-    return y;
-}
-
 // Outputs of one launch.  Scores modes: scores [n_rows, ld] (row r = query
 // row_begin + r; in the sampled mode column j is key j * kSampleStride) and
 // optional row_stats [n_rows, 8].  Candidate mode: tau [n_rows] (the row's
@@ -316,11 +294,9 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
     } else {
         // ------------------------------------------------------------ epilogue
         // Thread = one key of the tile (lane quarter qw), CW columns = QPW
-        // whole queries.  (Skipping the causal test on steps that lie wholly
-        // below the block, and the ReLU split between the two pipes, did not
-        // change the time at 128K: with every score stored, the stores and
-        // the math each cost about as much, and the MMA/TMEM pipeline below
-        // them sets a floor about 40 % lower.)
+        // whole queries.  The TMEM reads, the ReLU + head sum and the score
+        // stores (or the candidate ballot) each cost about as much at 128K;
+        // the MMA/TMA pipeline alone runs about 2.4x faster than the whole.
         const int qw = warp & 3;          // TMEM lane quarter: keys 32*qw ..
         const int cg = warp >> 2;         // column group: columns cg*CW ..
         const uint32_t lane_base = tmem_base + ((uint32_t)(qw * 32) << 16);
@@ -331,16 +307,13 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
             const int t0 = row_begin + qb * NQ;
             const int t_hi = min(t0 + NQ, row_end) - 1;
             const int nstep = (t_hi / KS) / kStepKeys + 1;
-            // this warp's query head weights, in registers for the whole
-            // block; the pairs that take the mul.sat ReLU are pre-scaled
+            // this warp's query head weights, in registers for the whole block
             float2 wv[CW / 2];
 #pragma unroll
             for (int c = 0; c < CW; c += 2) {
                 const int t = t0 + (cg * CW + c) / HI;
-                float2 x = t <= t_hi ? __ldg(reinterpret_cast<const float2 *>(w + (size_t)t0 * HI + cg * CW + c))
-                                     : make_float2(0.f, 0.f);
-                if (sat_pair(c / 2)) x = make_float2(x.x * kSatUp, x.y * kSatUp);
-                wv[c / 2] = x;
+                wv[c / 2] = t <= t_hi ? __ldg(reinterpret_cast<const float2 *>(w + (size_t)t0 * HI + cg * CW + c))
+                                      : make_float2(0.f, 0.f);
             }
             float sqv[QPW], vlo[QPW], vhi[QPW], tau[QPW];
             int cnt[QPW];
@@ -381,14 +354,12 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                             const int col = c * 32 + j;              // within this warp's CW columns
                             const int q = col / HI;                  // compile-time after unrolling
                             const int chain = (j >> 2) & 1;
-                            const float2 r0 = sat_pair(col / 2)
-                                                  ? make_float2(relu_sat(acc[j]), relu_sat(acc[j + 1]))
-                                                  : make_float2(fmaxf(acc[j], 0.f), fmaxf(acc[j + 1], 0.f));
-                            part[q][chain] = tc::ffma2(wv[col / 2], r0, part[q][chain]);
-                            const float2 r1 = sat_pair(col / 2 + 1)
-                                                  ? make_float2(relu_sat(acc[j + 2]), relu_sat(acc[j + 3]))
-                                                  : make_float2(fmaxf(acc[j + 2], 0.f), fmaxf(acc[j + 3], 0.f));
-                            part[q][chain] = tc::ffma2(wv[col / 2 + 1], r1, part[q][chain]);
+                            part[q][chain] = tc::ffma2(wv[col / 2],
+                                                       make_float2(fmaxf(acc[j], 0.f), fmaxf(acc[j + 1], 0.f)),
+                                                       part[q][chain]);
+                            part[q][chain] = tc::ffma2(wv[col / 2 + 1],
+                                                       make_float2(fmaxf(acc[j + 2], 0.f), fmaxf(acc[j + 3], 0.f)),
+                                                       part[q][chain]);
                         }
                     }
 #pragma unroll
