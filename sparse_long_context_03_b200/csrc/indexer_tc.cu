@@ -50,6 +50,27 @@ __device__ unsigned long long g_wait_limit_ns = 2000000000ull;
 
 namespace {
 
+// Pipeline waits with the bound above.  The bound is read only once a wait
+// has to spin (the barrier was not already complete), so it occupies no
+// register in the common case.
+__device__ __forceinline__ uint64_t pipe_wait_limit() {
+    return *const_cast<const volatile unsigned long long *>(&g_wait_limit_ns);
+}
+
+__device__ __forceinline__ bool pipe_wait(uint32_t bar, uint32_t parity) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    return tc::mbar_wait(bar, parity, pipe_wait_limit());
+}
+
+__device__ __forceinline__ bool pipe_wait_sleep(uint32_t bar, uint32_t parity, uint32_t sleep_ns) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    return tc::mbar_wait_sleep(bar, parity, pipe_wait_limit(), sleep_ns);
+}
+
+}  // namespace
+
+namespace {
+
 constexpr int kTileM = 128;     // keys per MMA (UMMA M)
 constexpr int kTileN = 128;     // (query, head) columns per tile
 constexpr int kStepKeys = 256;  // keys per pipeline step: two MMA tiles
@@ -118,7 +139,8 @@ enum IndexerMode : int {
 // threshold), cand [n_rows, 4, seg_cap] (index, score) pairs, one segment per
 // TMEM lane quarter, in ascending key order within a segment, and
 // cand_count [n_rows, 4] (the number of entries each segment would hold;
-// entries past seg_cap are dropped).
+// entries past seg_cap are dropped).  With packed sequences every key index
+// and output column is relative to the start of the query's sequence.
 struct EpiArgs {
     float *scores;
     int64_t ld;
@@ -127,9 +149,14 @@ struct EpiArgs {
     int2 *cand;
     int *cand_count;
     int seg_cap;
+    // packed sequences (VARLEN): query t sees the keys [start(t), t] of its
+    // own sequence, start(t) from cu [nseq + 1]; output columns and
+    // candidate indices are positions relative to start(t)
+    const int32_t *cu;
+    int nseq;
 };
 
-template <int HI, int DI, int MODE>
+template <int HI, int DI, int MODE, bool VARLEN>
 __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                                                  const __grid_constant__ CUtensorMap tmap_q,
                                                                  const float *__restrict__ sq,
@@ -164,7 +191,6 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
     const int warp = threadIdx.x >> 5, lane = lane_id();
     const int row_end = row_begin + n_rows;
     const int nb = (n_rows + NQ - 1) / NQ;
-    const uint64_t wait_ns = g_wait_limit_ns;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -207,16 +233,17 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                 const int t0 = row_begin + qb * NQ;
                 const int t_hi = min(t0 + NQ, row_end) - 1;
                 const int nstep = (t_hi / KS) / kStepKeys + 1;
+                const int st_lo = VARLEN ? ((seq_start(args.cu, args.nseq, t0) + KS - 1) / KS) / kStepKeys : 0;
                 const int qs = bi & 1;
-                if (!tc::mbar_wait_sleep(qempty_bar(qs), ((bi >> 1) & 1) ^ 1, wait_ns, kIssuerSleepNs)) {
+                if (!pipe_wait_sleep(qempty_bar(qs), ((bi >> 1) & 1) ^ 1, kIssuerSleepNs)) {
                     ok = false;
                     break;
                 }
                 tc::mbar_arrive_expect_tx(qfull_bar(qs), Lay::kQBytes);
                 tc::tma_load_2d(sbase + Lay::kQ + qs * Lay::kQBytes, &tmap_q, 0, t0 * HI, qfull_bar(qs));
                 ++q_issued;
-                for (int st = 0; st < nstep; ++st) {
-                    if (!tc::mbar_wait_sleep(empty_bar(stage), phase ^ 1, wait_ns, kIssuerSleepNs)) {
+                for (int st = st_lo; st < nstep; ++st) {
+                    if (!pipe_wait_sleep(empty_bar(stage), phase ^ 1, kIssuerSleepNs)) {
                         ok = false;
                         break;
                     }
@@ -251,20 +278,20 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                 const int t0 = row_begin + qb * NQ;
                 const int t_hi = min(t0 + NQ, row_end) - 1;
                 const int nstep = (t_hi / KS) / kStepKeys + 1;
+                const int st_lo = VARLEN ? ((seq_start(args.cu, args.nseq, t0) + KS - 1) / KS) / kStepKeys : 0;
                 const int qs = bi & 1;
-                if (!tc::mbar_wait_sleep(qfull_bar(qs), (bi >> 1) & 1, wait_ns, kIssuerSleepNs)) {
+                if (!pipe_wait_sleep(qfull_bar(qs), (bi >> 1) & 1, kIssuerSleepNs)) {
                     ok = false;
                     break;
                 }
                 tc::tc_fence_after();
                 const uint32_t qaddr = sbase + Lay::kQ + qs * Lay::kQBytes;
-                for (int st = 0; st < nstep; ++st, ++it) {
+                for (int st = st_lo; st < nstep; ++st, ++it) {
                     if ((it & 1) != mw) continue;
                     const int pr = mw;
                     const int stage = it % kStages;
-                    if (!tc::mbar_wait_sleep(tempty_bar(pr), ((it / kPairs) & 1) ^ 1, wait_ns,
-                                             kIssuerSleepNs) ||
-                        !tc::mbar_wait_sleep(full_bar(stage), (it / kStages) & 1, wait_ns, kIssuerSleepNs)) {
+                    if (!pipe_wait_sleep(tempty_bar(pr), ((it / kPairs) & 1) ^ 1, kIssuerSleepNs) ||
+                        !pipe_wait_sleep(full_bar(stage), (it / kStages) & 1, kIssuerSleepNs)) {
                         ok = false;
                         break;
                     }
@@ -307,6 +334,7 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
             const int t0 = row_begin + qb * NQ;
             const int t_hi = min(t0 + NQ, row_end) - 1;
             const int nstep = (t_hi / KS) / kStepKeys + 1;
+            const int st_lo = VARLEN ? ((seq_start(args.cu, args.nseq, t0) + KS - 1) / KS) / kStepKeys : 0;
             // this warp's query head weights, in registers for the whole block
             float2 wv[CW / 2];
 #pragma unroll
@@ -316,10 +344,11 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                                       : make_float2(0.f, 0.f);
             }
             float sqv[QPW], vlo[QPW], vhi[QPW], tau[QPW];
-            int cnt[QPW];
+            int cnt[QPW], jlo[QPW];  // jlo: first visible key (key-map units) of each query
 #pragma unroll
             for (int q = 0; q < QPW; ++q) {
                 const int t = t0 + (cg * CW) / HI + q;
+                jlo[q] = VARLEN && t <= t_hi ? (seq_start(args.cu, args.nseq, t) + KS - 1) / KS : 0;
                 sqv[q] = t <= t_hi ? __ldg(sq + t) : 0.f;
                 vlo[q] = INFINITY;
                 vhi[q] = -INFINITY;
@@ -327,9 +356,9 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                 if constexpr (MODE == kModeCand) tau[q] = t <= t_hi ? __ldg(args.tau + (t - row_begin)) : INFINITY;
                 else tau[q] = 0.f;
             }
-            for (int st = 0; st < nstep; ++st, ++it) {
+            for (int st = st_lo; st < nstep; ++st, ++it) {
                 const int pr = it % kPairs;
-                if (!tc::mbar_wait(tfull_bar(pr), (it / kPairs) & 1, wait_ns)) { ok = false; break; }
+                if (!pipe_wait(tfull_bar(pr), (it / kPairs) & 1)) { ok = false; break; }
                 tc::tc_fence_after();
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
@@ -365,7 +394,7 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
 #pragma unroll
                     for (int q = 0; q < QPW; ++q) {
                         const int t = t0 + (cg * CW) / HI + q;
-                        const bool vis = t <= t_hi && s * KS <= t;
+                        const bool vis = t <= t_hi && s * KS <= t && (!VARLEN || s >= jlo[q]);
                         if constexpr (MODE == kModeCand) {
                             // keep the scores at or above the row's threshold: warp-aggregated
                             // slots in this warp's own segment of the row (keys in ascending order)
@@ -377,13 +406,13 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
                                 const int pos = cnt[q] + __popc(b & ((1u << lane) - 1u));
                                 if (keep && pos < args.seg_cap)
                                     args.cand[((size_t)(t - row_begin) * 4 + qw) * args.seg_cap + pos] =
-                                        make_int2(s, __float_as_int(score));
+                                        make_int2(s - jlo[q], __float_as_int(score));
                                 cnt[q] += __popc(b);
                             }
                         } else if (vis) {
                             const float v = (part[q][0].x + part[q][1].x) + (part[q][0].y + part[q][1].y);
                             const float score = v * sqv[q] * sks;
-                            args.scores[(size_t)(t - row_begin) * args.ld + s] = score;
+                            args.scores[(size_t)(t - row_begin) * args.ld + (s - jlo[q])] = score;
                             if constexpr (MODE == kModeScores) {
                                 vlo[q] = fminf(vlo[q], score);
                                 vhi[q] = fmaxf(vhi[q], score);
@@ -888,7 +917,7 @@ cudaError_t set_smem_once(int smem) {
     return e;
 }
 
-template <int HI, int DI, int MODE>
+template <int HI, int DI, int MODE, bool VARLEN>
 cudaError_t launch_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8, const float *sk, int L,
                       int row_begin, int n_rows, const EpiArgs &a, cudaStream_t stream) {
     constexpr int KS = MODE == kModeSample ? kSampleStride : 1;
@@ -901,10 +930,10 @@ cudaError_t launch_tc(const uint8_t *q8, const float *sq, const float *w, const 
     const int grid = nb < sm_count() ? nb : sm_count();
     // at least 116 KB so that one CTA (and its 512 TMEM columns) owns each SM
     constexpr int smem = Layout<DI>::kAlloc > 116 * 1024 ? Layout<DI>::kAlloc : 116 * 1024;
-    cudaError_t e = set_smem_once<indexer_tc_kernel<HI, DI, MODE>>(smem);
+    cudaError_t e = set_smem_once<indexer_tc_kernel<HI, DI, MODE, VARLEN>>(smem);
     if (e != cudaSuccess) return e;
-    indexer_tc_kernel<HI, DI, MODE><<<grid, EpiShape<HI>::kThreads, smem, stream>>>(mk, mq, sq, w, sk, row_begin,
-                                                                                   n_rows, a);
+    indexer_tc_kernel<HI, DI, MODE, VARLEN><<<grid, EpiShape<HI>::kThreads, smem, stream>>>(mk, mq, sq, w, sk,
+                                                                                           row_begin, n_rows, a);
     return cudaGetLastError();
 }
 
@@ -936,12 +965,22 @@ cudaError_t launch_prefill_mode(const uint8_t *q8, const float *sq, const float 
                                 const float *sk, int L, int HI, int dI, int row_begin, int n_rows, const EpiArgs &a,
                                 cudaStream_t stream) {
     if (n_rows == 0) return cudaSuccess;
+    // packed sequences only on the fused path's modes (the scores mode keeps one sequence per call)
+    constexpr bool kVarlenModes = MODE != kModeScores;
     auto by_di = [&](auto hi) -> cudaError_t {
         constexpr int H = decltype(hi)::value;
+        if (kVarlenModes && a.cu != nullptr) {
+            switch (dI) {
+                case 32: return launch_tc<H, 32, MODE, kVarlenModes>(q8, sq, w, k8, sk, L, row_begin, n_rows, a, stream);
+                case 64: return launch_tc<H, 64, MODE, kVarlenModes>(q8, sq, w, k8, sk, L, row_begin, n_rows, a, stream);
+                case 128: return launch_tc<H, 128, MODE, kVarlenModes>(q8, sq, w, k8, sk, L, row_begin, n_rows, a, stream);
+                default: return cudaErrorInvalidValue;
+            }
+        }
         switch (dI) {
-            case 32: return launch_tc<H, 32, MODE>(q8, sq, w, k8, sk, L, row_begin, n_rows, a, stream);
-            case 64: return launch_tc<H, 64, MODE>(q8, sq, w, k8, sk, L, row_begin, n_rows, a, stream);
-            case 128: return launch_tc<H, 128, MODE>(q8, sq, w, k8, sk, L, row_begin, n_rows, a, stream);
+            case 32: return launch_tc<H, 32, MODE, false>(q8, sq, w, k8, sk, L, row_begin, n_rows, a, stream);
+            case 64: return launch_tc<H, 64, MODE, false>(q8, sq, w, k8, sk, L, row_begin, n_rows, a, stream);
+            case 128: return launch_tc<H, 128, MODE, false>(q8, sq, w, k8, sk, L, row_begin, n_rows, a, stream);
             default: return cudaErrorInvalidValue;
         }
     };
@@ -968,17 +1007,23 @@ cudaError_t launch_indexer_prefill_tc(const uint8_t *q8, const float *sq, const 
 
 cudaError_t launch_indexer_sample_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
                                      const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
-                                     float *sample_scores, int64_t ld, cudaStream_t stream) {
+                                     float *sample_scores, int64_t ld, const int32_t *cu, int nseq,
+                                     cudaStream_t stream) {
     EpiArgs a{};
     a.scores = sample_scores;
     a.ld = ld;
+    a.cu = cu;
+    a.nseq = nseq;
     return launch_prefill_mode<kModeSample>(q8, sq, w, k8, sk, L, HI, dI, row_begin, n_rows, a, stream);
 }
 
 cudaError_t launch_indexer_cand_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
                                    const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
-                                   const float *tau, int2 *cand, int *cand_count, int seg_cap, cudaStream_t stream) {
+                                   const float *tau, int2 *cand, int *cand_count, int seg_cap, const int32_t *cu,
+                                   int nseq, cudaStream_t stream) {
     EpiArgs a{};
+    a.cu = cu;
+    a.nseq = nseq;
     a.tau = tau;
     a.cand = cand;
     a.cand_count = cand_count;
