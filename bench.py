@@ -461,6 +461,54 @@ def run_kl_timed(dsa, inputs, pk, reps=5, n_rows=4096, G=4):
     return out
 
 
+def run_packed_timed(dsa, inputs, steps, warmup, lens=None):
+    """Packed (varlen) prefill: 64 sequences of 2K tokens and 4 of 32K in one
+    token axis, every stage one launch over all of them
+    (dsa_indexer_topk_varlen, dsa_sparse_gqa_prefill_varlen).  Returns
+    tokens/s and the stage times, CUDA events on the launch stream."""
+    cfg = inputs.config(1)
+    lens = lens or [2048] * 64 + [32768] * 4
+    cu = torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32, device="cuda")
+    total = int(cu[-1].item())
+    d = inputs.prefill_inputs(cfg, device="cuda", L=total, seed=cfg.seed + 17)
+    plan = dsa.PrefillPlan(total, cfg.HI, cfg.dI, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, device="cuda", fused=True)
+    O = torch.empty(total, cfg.Hq, cfg.D, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        a = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for r0, n in plan.chunks():
+            dsa.indexer_topk_varlen(d["q8"], d["sq"], d["w"], d["k8"], d["sk"], cu, r0, n, cfg.k,
+                                    plan.idx[r0:r0 + n], plan.ws)
+        b = torch.cuda.Event(enable_timing=True)
+        b.record(stream)
+        dsa.sparse_gqa_prefill_varlen(d["Q"], d["K"], d["V"], plan.idx, cu, 0, total, cfg.k, cfg.sm_scale, O)
+        c = torch.cuda.Event(enable_timing=True)
+        c.record(stream)
+        if ev is not None:
+            ev.append((a, b, c))
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = []
+    for _ in range(steps):
+        step(ev)
+    torch.cuda.synchronize()
+    dsa.check_device_error()
+    sel = sum(a.elapsed_time(b) for a, b, _ in ev) / steps
+    att = sum(b.elapsed_time(c) for _, b, c in ev) / steps
+    ms = sel + att
+    pairs = sum(n * (n + 1) // 2 for n in lens)
+    return {"workload": f"packed prefill: {len(lens)} sequences ({lens.count(2048)} x 2048 + "
+                        f"{lens.count(32768)} x 32768 tokens, {total} in all), layer as prefill-32k",
+            "value": total / (ms / 1e3), "unit": "tok/s", "ms_per_step": ms, "steps": steps,
+            "stages_ms": {"indexer_topk_varlen": sel, "attention_varlen": att},
+            "indexer_tflops": 2 * cfg.HI * cfg.dI * pairs / (sel / 1e3) / 1e12,
+            "launches_per_step": 5 * len(list(plan.chunks())) + 1}
+
+
 class DecodeBench:
     def __init__(self, cfg, seed, device, batch=None):
         from sparse_long_context_03_b200 import dsa, inputs
@@ -745,6 +793,7 @@ def main():
     ap.add_argument("--chunk-rows", type=int, default=None,
                     help="query rows per indexer/top-k chunk (default: a 4 GiB score block)")
     ap.add_argument("--no-kl", action="store_true", help="skip the indexer distillation-loss leg")
+    ap.add_argument("--no-packed", action="store_true", help="skip the packed (varlen) prefill leg")
     ap.add_argument("--unfused", action="store_true",
                     help="materialise the score matrix per chunk and run dsa_topk (instead of dsa_indexer_topk)")
     ap.add_argument("--decode-batch", type=int, default=None,
@@ -821,6 +870,12 @@ def main():
         torch.cuda.empty_cache()
         pb = None
 
+    packed = None
+    if rank == 0 and not args.no_packed:
+        from sparse_long_context_03_b200 import dsa as _dsa_pk
+        packed = run_packed_timed(_dsa_pk, inputs, max(args.steps, 3), max(args.warmup, 1))
+        torch.cuda.empty_cache()
+
     kl = None
     if rank == 0 and not args.no_kl:
         from sparse_long_context_03_b200 import dsa as _dsa_kl
@@ -848,7 +903,7 @@ def main():
                              "candidate lists or 4 GiB score chunks)"},
             "roofline": dom_line, "stages": stages, "clocks": clocks, "gpu_launches": None,
             "peaks_measured_here": {"fp8": fp8, "reads": reads},
-            "e2e": e2e, "decode": decode, "indexer_kl": kl, "cpu_baseline": cpu,
+            "e2e": e2e, "decode": decode, "packed": packed, "indexer_kl": kl, "cpu_baseline": cpu,
         }
         # kernels per library call: the fused threshold stage runs the sampled indexer and the threshold
         # select, the select stage the candidate select, the repair kernel and the stats copy

@@ -177,6 +177,23 @@ DSA_API dsa_status_t dsa_indexer_topk(const uint8_t *q8, const float *q_scale, c
                               const uint8_t *k8, const float *k_scale,
                               int L, int HI, int dI, int row_begin, int n_rows, int k,
                               int32_t *idx, void *ws, size_t ws_bytes, int64_t *stats, void *stream);
+/* Packed (varlen) form of dsa_indexer_topk: several sequences packed along
+ * the token axis, each its own causal prefill ([REPORT] 5.1.2: per-sample
+ * causal regions in one launch).  Sequence b holds tokens
+ * cu_seqlens[b] .. cu_seqlens[b+1]-1; query token t of sequence b scores and
+ * selects only the keys cu_seqlens[b] .. t, and idx row r (t = row_begin +
+ * r) holds positions within that sequence (0 = its first token), ascending,
+ * -1 padded; a row with t - cu_seqlens[b] + 1 <= k keeps all of them.
+ *   cu_seqlens  device int32 [nseq + 1], ascending, cu_seqlens[0] = 0,
+ *               cu_seqlens[nseq] = L (empty sequences allowed); read on the
+ *               device (a malformed array gives wrong rows, never reads
+ *               outside the tokens 0..t).
+ *   L           total packed tokens; every other argument as for
+ *               dsa_indexer_topk, with the same workspace size query. */
+DSA_API dsa_status_t dsa_indexer_topk_varlen(const uint8_t *q8, const float *q_scale, const float *w,
+                              const uint8_t *k8, const float *k_scale, int L, int HI, int dI,
+                              const int32_t *cu_seqlens, int nseq, int row_begin, int n_rows, int k,
+                              int32_t *idx, void *ws, size_t ws_bytes, int64_t *stats, void *stream);
 /* The three stages of dsa_indexer_topk, same arguments, for callers that time
  * or schedule them separately; called in this order on one stream, with the
  * same workspace and arguments, they are dsa_indexer_topk:
@@ -248,6 +265,16 @@ DSA_API dsa_status_t dsa_indexer_kl(const float *scores, int64_t ld_scores, int 
 DSA_API dsa_status_t dsa_sparse_gqa_prefill(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                                     const int32_t *idx, int row_begin, int n_rows,
                                     int Hq, int Hkv, int D, int k, float sm_scale,
+                                    uint16_t *O, float *lse, void *stream);
+/* Packed (varlen) form: sequence b holds tokens cu_seqlens[b] ..
+ * cu_seqlens[b+1]-1 (cu_seqlens as for dsa_indexer_topk_varlen, device int32
+ * [nseq + 1]); idx row r (query t = row_begin + r of sequence b) holds
+ * positions within sequence b, and entry e names token cu_seqlens[b] + e;
+ * entries outside [0, t - cu_seqlens[b]] are skipped.  Q, O rows and K, V
+ * rows are packed tokens. */
+DSA_API dsa_status_t dsa_sparse_gqa_prefill_varlen(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                                    const int32_t *idx, const int32_t *cu_seqlens, int nseq,
+                                    int row_begin, int n_rows, int Hq, int Hkv, int D, int k, float sm_scale,
                                     uint16_t *O, float *lse, void *stream);
 
 /* ------------------------------------------------------------------------

@@ -139,7 +139,8 @@ namespace {
 dsa_status_t indexer_topk_checked(int stage, const uint8_t *q8, const float *q_scale, const float *w,
                                   const uint8_t *k8, const float *k_scale, int L, int HI, int dI, int row_begin,
                                   int n_rows, int k, int32_t *idx, void *ws, size_t ws_bytes, int64_t *stats,
-                                  void *stream) {
+                                  void *stream, const int32_t *cu = nullptr, int nseq = 0) {
+    if (cu != nullptr && nseq < 1) return DSA_ERR_INVALID_ARG;
     if (L < 1 || row_begin < 0 || n_rows < 0 || k < 1 || (int64_t)row_begin + n_rows > L) return DSA_ERR_INVALID_ARG;
     if (!dsa::fused_topk_supported(k, HI, dI) || (int64_t)L * HI >= (1ll << 31)) return DSA_ERR_UNSUPPORTED_SHAPE;
     if (n_rows == 0) return DSA_OK;
@@ -149,7 +150,7 @@ dsa_status_t indexer_topk_checked(int stage, const uint8_t *q8, const float *q_s
     if (ws == nullptr || ws_bytes < need || reinterpret_cast<uintptr_t>(ws) % 256 != 0) return DSA_ERR_WORKSPACE;
     for (int st = stage == 0 ? 1 : stage; st <= (stage == 0 ? 3 : stage); ++st) {
         const cudaError_t e = dsa::launch_indexer_topk_stage(st, q8, q_scale, w, k8, k_scale, L, HI, dI, row_begin,
-                                                             n_rows, k, idx, ws, stats, as_stream(stream));
+                                                             n_rows, k, idx, ws, stats, cu, nseq, as_stream(stream));
         if (e != cudaSuccess) return cuda_status(e);
     }
     return DSA_OK;
@@ -165,6 +166,16 @@ dsa_status_t dsa_indexer_topk(const uint8_t *q8, const float *q_scale, const flo
     const Range range(__func__);
     return indexer_topk_checked(0, q8, q_scale, w, k8, k_scale, L, HI, dI, row_begin, n_rows, k, idx, ws, ws_bytes,
                                 stats, stream);
+}
+
+dsa_status_t dsa_indexer_topk_varlen(const uint8_t *q8, const float *q_scale, const float *w, const uint8_t *k8,
+                                     const float *k_scale, int L, int HI, int dI, const int32_t *cu_seqlens, int nseq,
+                                     int row_begin, int n_rows, int k, int32_t *idx, void *ws, size_t ws_bytes,
+                                     int64_t *stats, void *stream) {
+    const Range range(__func__);
+    if (cu_seqlens == nullptr) return DSA_ERR_INVALID_ARG;
+    return indexer_topk_checked(0, q8, q_scale, w, k8, k_scale, L, HI, dI, row_begin, n_rows, k, idx, ws, ws_bytes,
+                                stats, stream, cu_seqlens, nseq);
 }
 
 dsa_status_t dsa_indexer_topk_threshold(const uint8_t *q8, const float *q_scale, const float *w, const uint8_t *k8,
@@ -216,6 +227,21 @@ dsa_status_t dsa_sparse_gqa_prefill(const uint16_t *Q, const uint16_t *K, const 
     if (!Q || !K || !V || !idx || !O) return DSA_ERR_INVALID_ARG;
     return cuda_status(dsa::launch_sparse_prefill(Q, K, V, idx, row_begin, n_rows, Hq, Hkv, D, k, sm_scale, O, lse,
                                                   as_stream(stream)));
+}
+
+dsa_status_t dsa_sparse_gqa_prefill_varlen(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                                           const int32_t *idx, const int32_t *cu_seqlens, int nseq, int row_begin,
+                                           int n_rows, int Hq, int Hkv, int D, int k, float sm_scale, uint16_t *O,
+                                           float *lse, void *stream) {
+    const Range range(__func__);
+    if (cu_seqlens == nullptr || nseq < 1) return DSA_ERR_INVALID_ARG;
+    if (row_begin < 0 || n_rows < 0 || k < 1 || Hq < 1 || Hkv < 1) return DSA_ERR_INVALID_ARG;
+    if (!dsa::attention_shape_supported(Hq, Hkv, D)) return DSA_ERR_UNSUPPORTED_SHAPE;
+    if ((int64_t)n_rows * Hkv >= (1ll << 31)) return DSA_ERR_UNSUPPORTED_SHAPE;  // one CTA per (row, group)
+    if (n_rows == 0) return DSA_OK;
+    if (!Q || !K || !V || !idx || !O) return DSA_ERR_INVALID_ARG;
+    return cuda_status(dsa::launch_sparse_prefill(Q, K, V, idx, row_begin, n_rows, Hq, Hkv, D, k, sm_scale, O, lse,
+                                                  as_stream(stream), cu_seqlens, nseq));
 }
 
 // The decode indexer copies cache pages and query rows in 16-byte pieces.

@@ -231,7 +231,7 @@ template <int D>
 __global__ void __launch_bounds__(kWarpsPerCta * 32) sparse_prefill_kernel(
     const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K, const uint16_t *__restrict__ V,
     const int32_t *__restrict__ idx, int row_begin, int n_rows, int Hq, int Hkv, int k, float scale_log2,
-    uint16_t *__restrict__ O, float *__restrict__ lse, int group_major) {
+    uint16_t *__restrict__ O, float *__restrict__ lse, int group_major, const int32_t *__restrict__ cu, int nseq) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = lane_id();
     const int pair = blockIdx.x * kWarpsPerCta + warp;
@@ -246,10 +246,16 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) sparse_prefill_kernel(
 
     WarpAttn<D> st;
     load_q<D>(st, Q + ((size_t)r * Hq + (size_t)g * G) * D, G, lane);
-    const int n_vis = min(k, t + 1);
+    // packed sequences: row t attends to positions 0..t-start of its own
+    // sequence, i.e. tokens start..t (start = 0 for a single sequence)
+    const int start = seq_start(cu, nseq, t);
+    const int n_vis = min(k, t - start + 1);
     attend_range<D>(
         st, wsmem, idx + (size_t)r * k, 0, n_vis, K, V, scale_log2,
-        [&](int32_t s) -> int64_t { return (s >= 0 && s <= t) ? ((int64_t)s * Hkv + g) * D : -1; }, lane);
+        [&](int32_t s) -> int64_t {
+            return (s >= 0 && s <= t - start) ? ((int64_t)(start + s) * Hkv + g) * D : -1;
+        },
+        lane);
     reduce_sums<D>(st);
 
     // Normalise, stage the group's [G, D] output tile in shared memory, then
@@ -394,7 +400,7 @@ bool attention_shape_supported(int Hq, int Hkv, int D) {
 
 cudaError_t launch_sparse_prefill(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const int32_t *idx,
                                   int row_begin, int n_rows, int Hq, int Hkv, int D, int k, float sm_scale,
-                                  uint16_t *O, float *lse, cudaStream_t stream) {
+                                  uint16_t *O, float *lse, cudaStream_t stream, const int32_t *cu, int nseq) {
     if (n_rows == 0) return cudaSuccess;
     const int64_t pairs = (int64_t)n_rows * Hkv;
     const int grid = (int)((pairs + kWarpsPerCta - 1) / kWarpsPerCta);
@@ -410,7 +416,7 @@ cudaError_t launch_sparse_prefill(const uint16_t *Q, const uint16_t *K, const ui
         if (err != cudaSuccess) return true;
         sparse_prefill_kernel<DD><<<grid, kWarpsPerCta * 32, smem, stream>>>(Q, K, V, idx, row_begin, n_rows, Hq,
                                                                              Hkv, k, sm_scale * kLog2e, O, lse,
-                                                                             group_major ? 1 : 0);
+                                                                             group_major ? 1 : 0, cu, nseq);
         err = cudaGetLastError();
         return true;
     });

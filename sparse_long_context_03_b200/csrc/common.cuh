@@ -106,6 +106,25 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // ---------------------------------------------------------------------------
+// Packed (varlen) sequences
+// ---------------------------------------------------------------------------
+
+// First token of the packed sequence that holds token t: cu[b] for the
+// largest b < nseq with cu[b] <= t, where cu [nseq + 1] is ascending with
+// cu[0] = 0 (empty sequences allowed).  0 without cu.  Clamped to [0, t], so
+// that a malformed cu cannot send a read outside the tokens 0..t.
+__device__ __forceinline__ int seq_start(const int32_t *cu, int nseq, int t) {
+    if (cu == nullptr || nseq < 1) return 0;
+    int lo = 0, hi = nseq;  // the answer lies in [lo, hi)
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(cu + mid) <= t) lo = mid; else hi = mid;
+    }
+    const int s = __ldg(cu + lo);
+    return s < 0 ? 0 : (s > t ? t : s);
+}
+
+// ---------------------------------------------------------------------------
 // Top-k keys
 // ---------------------------------------------------------------------------
 

@@ -28,16 +28,20 @@ cudaError_t indexer_tc_take_error(unsigned int *flag);
 // bound of the prefill indexer's pipeline waits on the current device (0: the default)
 cudaError_t indexer_tc_set_wait_limit(unsigned long long ns);
 // the same kernel scoring every indexer_sample_stride()-th key only:
-// sample_scores [n_rows, ld], column j = key j * stride (causal: j * stride <= t)
+// sample_scores [n_rows, ld], column j = key j * stride (causal: j * stride <= t);
+// with cu (packed sequences, cu [nseq + 1]) the keys of the query's own
+// sequence only, column j = the j-th sampled key at or after its start
 int indexer_sample_stride();
 cudaError_t launch_indexer_sample_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
                                      const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
-                                     float *sample_scores, int64_t ld, cudaStream_t stream);
+                                     float *sample_scores, int64_t ld, const int32_t *cu, int nseq,
+                                     cudaStream_t stream);
 // the same kernel keeping only scores >= tau[row]: (index, score) pairs in
 // cand [n_rows, 4, seg_cap], counts (uncapped) in cand_count [n_rows, 4]
 cudaError_t launch_indexer_cand_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8,
                                    const float *sk, int L, int HI, int dI, int row_begin, int n_rows,
-                                   const float *tau, int2 *cand, int *cand_count, int seg_cap, cudaStream_t stream);
+                                   const float *tau, int2 *cand, int *cand_count, int seg_cap, const int32_t *cu,
+                                   int nseq, cudaStream_t stream);
 bool indexer_decode_tc_supported(int HI, int dI, int B, int max_seq_len);
 cudaError_t launch_indexer_decode_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8c,
                                      const float *skc, const int32_t *block_table, int max_pages, int num_pages,
@@ -69,7 +73,7 @@ bool fused_topk_supported(int k, int HI, int dI);
 cudaError_t launch_indexer_topk_stage(int stage, const uint8_t *q8, const float *sq, const float *w,
                                       const uint8_t *k8, const float *sk, int L, int HI, int dI, int row_begin,
                                       int n_rows, int k, int32_t *idx, void *ws, int64_t *stats,
-                                      cudaStream_t stream);
+                                      const int32_t *cu, int nseq, cudaStream_t stream);
 
 // indexer_kl.cu: the indexer's distillation losses (forward)
 cudaError_t launch_indexer_kl(const float *scores, int64_t ld, int row_begin, int n_rows, const float *p, int G,
@@ -78,9 +82,12 @@ cudaError_t launch_indexer_kl(const float *scores, int64_t ld, int row_begin, in
 
 // attention.cu
 bool attention_shape_supported(int Hq, int Hkv, int D);
+// cu [nseq + 1] (optional): packed sequences; index rows hold positions
+// within each query's own sequence
 cudaError_t launch_sparse_prefill(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const int32_t *idx,
                                   int row_begin, int n_rows, int Hq, int Hkv, int D, int k, float sm_scale,
-                                  uint16_t *O, float *lse, cudaStream_t stream);
+                                  uint16_t *O, float *lse, cudaStream_t stream, const int32_t *cu = nullptr,
+                                  int nseq = 0);
 size_t decode_attention_workspace_bytes(int B, int Hq, int Hkv, int D, int k);
 cudaError_t launch_sparse_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
                                  const int32_t *block_table, int max_pages, int num_pages, const int32_t *seq_lens,

@@ -32,6 +32,10 @@
 //      radix path.  With no listed rows it exits at once.
 // Only step 2's threshold is sampled; the counts that decide each row are
 // exact, so the result does not depend on the sample.
+//
+// Packed sequences (cu [nseq + 1], optional): row t sees only the keys
+// [start(t), t] of its own sequence, and every index is a position within
+// that sequence.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -62,7 +66,8 @@ __global__ void __launch_bounds__(kThreads) sample_threshold_kernel(const float 
                                                                    int row_begin, int n_rows, int k, int keep_all,
                                                                    int stride, float *__restrict__ tau,
                                                                    int *__restrict__ repair,
-                                                                   unsigned long long *__restrict__ cand_total) {
+                                                                   unsigned long long *__restrict__ cand_total,
+                                                                   const int32_t *__restrict__ cu, int nseq) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     ThreshSmem &sm = *reinterpret_cast<ThreshSmem *>(smem_raw);
     const int r = blockIdx.x, tid = threadIdx.x;
@@ -71,12 +76,13 @@ __global__ void __launch_bounds__(kThreads) sample_threshold_kernel(const float 
         *cand_total = 0ull;
     }
     const int t = row_begin + r;
-    const int n = t + 1;
+    const int start = seq_start(cu, nseq, t);
+    const int n = t - start + 1;
     if (n <= keep_all) {
         if (tid == 0) tau[r] = -INFINITY;
         return;
     }
-    const int m = t / stride + 1;  // sampled keys visible to row t
+    const int m = t / stride - (start + stride - 1) / stride + 1;  // sampled keys visible to row t
     const float mu = (float)k * (float)m / (float)n;
     const int rsel = (int)ceilf(mu + 7.f * sqrtf(mu) + 8.f);
     if (rsel >= m) {
@@ -191,12 +197,13 @@ __global__ void __launch_bounds__(kThreads) cand_select_kernel(const int2 *__res
                                                               const int *__restrict__ cand_count, int seg_cap,
                                                               int row_begin, int k, int32_t *__restrict__ idx,
                                                               int *__restrict__ repair,
-                                                              unsigned long long *__restrict__ cand_total) {
+                                                              unsigned long long *__restrict__ cand_total,
+                                                              const int32_t *__restrict__ cu, int nseq) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     SelectSmem &sm = *reinterpret_cast<SelectSmem *>(smem_raw);
     const int r = blockIdx.x, tid = threadIdx.x;
     const int t = row_begin + r;
-    const int n = t + 1;
+    const int n = t - seq_start(cu, nseq, t) + 1;  // keys visible to row t (positions 0..n-1 of its sequence)
     int32_t *out = idx + (size_t)r * k;
     if (n <= k) {  // short row: everything visible is selected
         for (int i = tid; i < k; i += kThreads) out[i] = i < n ? i : -1;
@@ -443,7 +450,8 @@ constexpr int kRepairHeads = 8;  // heads accumulated at a time
 __global__ void __launch_bounds__(kRepairThreads) repair_rows_kernel(
     const uint8_t *__restrict__ q8, const float *__restrict__ sq, const float *__restrict__ w,
     const uint8_t *__restrict__ k8, const float *__restrict__ sk, int HI, int dI, int row_begin, int k,
-    const int *__restrict__ repair, float *__restrict__ scratch, int64_t scratch_ld, int32_t *__restrict__ idx) {
+    const int *__restrict__ repair, float *__restrict__ scratch, int64_t scratch_ld, int32_t *__restrict__ idx,
+    const int32_t *__restrict__ cu, int nseq) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
     float *qf = reinterpret_cast<float *>(smem_raw + (sizeof(TopkSmem) + 15) / 16 * 16);  // [HI * dI]
@@ -453,7 +461,8 @@ __global__ void __launch_bounds__(kRepairThreads) repair_rows_kernel(
     for (int j = blockIdx.x; j < n_rep; j += gridDim.x) {
         const int r = __ldg(repair + 1 + j);
         const int t = row_begin + r;
-        const int n = t + 1;
+        const int start = seq_start(cu, nseq, t);
+        const int n = t - start + 1;
         for (int i = threadIdx.x; i < HI * dI / 2; i += kRepairThreads) {
             const uint16_t v = reinterpret_cast<const uint16_t *>(q8 + (size_t)t * HI * dI)[i];
             const float2 f = e4m3x2_to_float2(v);
@@ -463,7 +472,8 @@ __global__ void __launch_bounds__(kRepairThreads) repair_rows_kernel(
         for (int i = threadIdx.x; i < HI; i += kRepairThreads) wf[i] = __ldg(w + (size_t)t * HI + i);
         __syncthreads();
         const float sqt = __ldg(sq + t);
-        for (int s = threadIdx.x; s < n; s += kRepairThreads) {
+        for (int i = threadIdx.x; i < n; i += kRepairThreads) {
+            const int s = start + i;
             const uint16_t *kr = reinterpret_cast<const uint16_t *>(k8 + (size_t)s * dI);
             float acc = 0.f;
             for (int h0 = 0; h0 < HI; h0 += kRepairHeads) {
@@ -482,7 +492,7 @@ __global__ void __launch_bounds__(kRepairThreads) repair_rows_kernel(
 #pragma unroll
                 for (int j2 = 0; j2 < kRepairHeads; ++j2) acc = fmaf(wf[h0 + j2], fmaxf(d[j2], 0.f), acc);
             }
-            row[s] = acc * sqt * __ldg(sk + s);
+            row[i] = acc * sqt * __ldg(sk + s);
         }
         __syncthreads();
         topk_row_radix<true>(row, n, k, idx + (size_t)r * k, sm);
@@ -595,7 +605,7 @@ FusedPtrs fused_ptrs(const FusedTopkLayout &lay, void *ws) {
 cudaError_t launch_indexer_topk_stage(int stage, const uint8_t *q8, const float *sq, const float *w,
                                       const uint8_t *k8, const float *sk, int L, int HI, int dI, int row_begin,
                                       int n_rows, int k, int32_t *idx, void *ws, int64_t *stats,
-                                      cudaStream_t stream) {
+                                      const int32_t *cu, int nseq, cudaStream_t stream) {
     if (n_rows == 0) return cudaSuccess;
     const FusedTopkLayout lay = fused_topk_layout(row_begin, n_rows, k, HI, dI);
     const FusedPtrs P = fused_ptrs(lay, ws);
@@ -606,7 +616,7 @@ cudaError_t launch_indexer_topk_stage(int stage, const uint8_t *q8, const float 
         const int s0 = row_begin > lay.keep_all ? row_begin : lay.keep_all;
         if (s0 < row_end) {
             e = launch_indexer_sample_tc(q8, sq, w, k8, sk, L, HI, dI, s0, row_end - s0,
-                                         P.sample + (size_t)(s0 - row_begin) * lay.lds, lay.lds, stream);
+                                         P.sample + (size_t)(s0 - row_begin) * lay.lds, lay.lds, cu, nseq, stream);
             if (e != cudaSuccess) return e;
         }
         // thresholds (and the repair list emptied)
@@ -614,7 +624,7 @@ cudaError_t launch_indexer_topk_stage(int stage, const uint8_t *q8, const float 
         if (e != cudaSuccess) return e;
         sample_threshold_kernel<<<n_rows, kThreads, sizeof(ThreshSmem), stream>>>(
             P.sample, lay.lds, row_begin, n_rows, k, lay.keep_all, indexer_sample_stride(), P.tau, P.repair,
-            P.cand_total);
+            P.cand_total, cu, nseq);
         return cudaGetLastError();
     }
     if (stage == 2) {
@@ -623,7 +633,7 @@ cudaError_t launch_indexer_topk_stage(int stage, const uint8_t *q8, const float 
         if (c0 >= row_end) return cudaSuccess;
         return launch_indexer_cand_tc(q8, sq, w, k8, sk, L, HI, dI, c0, row_end - c0, P.tau + (c0 - row_begin),
                                       P.cand + (size_t)(c0 - row_begin) * kSegs * lay.seg_cap,
-                                      P.counts + (size_t)(c0 - row_begin) * kSegs, lay.seg_cap, stream);
+                                      P.counts + (size_t)(c0 - row_begin) * kSegs, lay.seg_cap, cu, nseq, stream);
     }
     if (stage == 3) {
         // exact selection, then the repair of the listed rows (which exits at
@@ -631,12 +641,12 @@ cudaError_t launch_indexer_topk_stage(int stage, const uint8_t *q8, const float 
         e = set_smem<cand_select_kernel>(lay.select_smem);
         if (e != cudaSuccess) return e;
         cand_select_kernel<<<n_rows, kThreads, lay.select_smem, stream>>>(P.cand, P.counts, lay.seg_cap, row_begin,
-                                                                          k, idx, P.repair, P.cand_total);
+                                                                          k, idx, P.repair, P.cand_total, cu, nseq);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         e = set_smem<repair_rows_kernel>(lay.repair_smem);
         if (e != cudaSuccess) return e;
         repair_rows_kernel<<<lay.repair_ctas, kRepairThreads, lay.repair_smem, stream>>>(
-            q8, sq, w, k8, sk, HI, dI, row_begin, k, P.repair, P.scratch, lay.scratch_ld, idx);
+            q8, sq, w, k8, sk, HI, dI, row_begin, k, P.repair, P.scratch, lay.scratch_ld, idx, cu, nseq);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if (stats != nullptr) {
             fused_stats_kernel<<<1, 1, 0, stream>>>(P.repair, P.cand_total, stats);

@@ -40,6 +40,8 @@ _SIGNATURES = {
     "dsa_topk": ([_P, _I64, _I, _I, _P, _I, _I, _P, _P, _P, _SZ, _P], _I),
     "dsa_indexer_topk_workspace_size": ([_I, _I, _I, _I, _I], _SZ),
     "dsa_indexer_topk": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P, _P], _I),
+    "dsa_indexer_topk_varlen": ([_P, _P, _P, _P, _P, _I, _I, _I, _P, _I, _I, _I, _I, _P, _P, _SZ, _P, _P], _I),
+    "dsa_sparse_gqa_prefill_varlen": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P], _I),
     "dsa_indexer_topk_threshold": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P, _P], _I),
     "dsa_indexer_topk_candidates": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P, _P], _I),
     "dsa_indexer_topk_select": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P, _P], _I),
@@ -235,6 +237,37 @@ def sparse_gqa_prefill(Q, K, V, idx, row_begin, n_rows, k, sm_scale, O, lse=None
            "dsa_sparse_gqa_prefill")
 
 
+def indexer_topk_varlen(q8, q_scale, w, k8, k_scale, cu_seqlens, row_begin, n_rows, k, idx, ws, stats=None,
+                        stream=None):
+    """dsa_indexer_topk_varlen: Omega_t of packed query rows [row_begin,
+    row_begin+n_rows); cu_seqlens int32 CUDA tensor [nseq+1].  idx [n_rows,
+    k] receives positions within each query's own sequence."""
+    _need(q8, torch.uint8, 3, "q8")
+    _need(k8, torch.uint8, 2, "k8")
+    _need(idx, torch.int32, 2, "idx")
+    _need(cu_seqlens, torch.int32, 1, "cu_seqlens")
+    L, HI, dI = q8.shape
+    _check(lib().dsa_indexer_topk_varlen(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), L, HI, dI,
+                                         _ptr(cu_seqlens), cu_seqlens.numel() - 1, int(row_begin), int(n_rows), int(k),
+                                         _ptr(idx), _ptr(ws), ws.numel() * ws.element_size(), _ptr(stats),
+                                         _stream(stream)), "dsa_indexer_topk_varlen")
+
+
+def sparse_gqa_prefill_varlen(Q, K, V, idx, cu_seqlens, row_begin, n_rows, k, sm_scale, O, lse=None, stream=None):
+    """dsa_sparse_gqa_prefill_varlen: attention of packed query rows over
+    their selected positions (relative to each query's own sequence)."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (O, "O")):
+        _need(t, torch.bfloat16, 3, n)
+    _need(idx, torch.int32, 2, "idx")
+    _need(cu_seqlens, torch.int32, 1, "cu_seqlens")
+    Hq, D = Q.shape[1], Q.shape[2]
+    Hkv = K.shape[1]
+    _check(lib().dsa_sparse_gqa_prefill_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(cu_seqlens),
+                                               cu_seqlens.numel() - 1, int(row_begin), int(n_rows), Hq, Hkv, D,
+                                               int(k), float(sm_scale), _ptr(O), _ptr(lse), _stream(stream)),
+           "dsa_sparse_gqa_prefill_varlen")
+
+
 class PrefillPlan:
     """Buffers for a prefill of one sequence.
 
@@ -311,20 +344,38 @@ def prefill_forward(plan: PrefillPlan, q8, sq, w, k8, sk, Q, K, V, O, sm_scale=N
 def prefill_forward_packed(plan: PrefillPlan, cu_seqlens, q8, sq, w, k8, sk, Q, K, V, O, sm_scale=None, lse=None,
                            idx_out=None, stream=None):
     """DSA prefill of several sequences packed along the token axis: sequence
-    b holds tokens cu_seqlens[b] .. cu_seqlens[b+1]-1 (host ints, ascending)
-    and is its own causal prefill -- no query scores or attends a key of
-    another sequence.  Every per-token tensor (q8, sq, w, k8, sk, Q, K, V, O,
-    lse) is indexed by the packed token; the chain runs on each sequence's
-    slice, so `plan` must be sized for the longest sequence.  idx_out, if
-    given, [total, k] int32, receives each token's selected positions within
-    its own sequence."""
-    cu = [int(x) for x in cu_seqlens]
+    b holds tokens cu_seqlens[b] .. cu_seqlens[b+1]-1 and is its own causal
+    prefill -- no query scores or attends a key of another sequence.  Every
+    per-token tensor (q8, sq, w, k8, sk, Q, K, V, O, lse) is indexed by the
+    packed token.  idx_out, if given, [total, k] int32, receives each token's
+    selected positions within its own sequence.
+
+    With the fused indexer + top-k (plan.fused; the plan sized for the
+    packed total), every stage is one launch per chunk of packed rows over
+    all sequences at once (dsa_indexer_topk_varlen,
+    dsa_sparse_gqa_prefill_varlen; cu_seqlens as a host sequence or an int32
+    CUDA tensor).  Otherwise (HI = 4) the score-matrix chain runs once per
+    sequence on its slice (cu_seqlens host ints; the plan sized for the
+    longest sequence)."""
+    cu = [int(x) for x in (cu_seqlens.tolist() if isinstance(cu_seqlens, torch.Tensor) else cu_seqlens)]
     if any(b < a for a, b in zip(cu, cu[1:])) or (cu and cu[0] != 0):
         raise DSAError("cu_seqlens must start at 0 and be non-decreasing")
-    if max((b - a for a, b in zip(cu, cu[1:])), default=0) > plan.L:
-        raise DSAError("a sequence is longer than the plan")
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(plan.D)
+    total = cu[-1] if cu else 0
+    if plan.fused:
+        if total > plan.L:
+            raise DSAError("the packed tokens exceed the plan")
+        cu_dev = cu_seqlens if isinstance(cu_seqlens, torch.Tensor) and cu_seqlens.is_cuda else \
+            torch.tensor(cu, dtype=torch.int32, device=q8.device)
+        idx = plan.idx[:total] if idx_out is None else idx_out
+        for r0 in range(0, total, plan.chunk_rows):
+            n = min(plan.chunk_rows, total - r0)
+            indexer_topk_varlen(q8, sq, w, k8, sk, cu_dev, r0, n, plan.k, idx[r0:r0 + n], plan.ws, stream=stream)
+        sparse_gqa_prefill_varlen(Q, K, V, idx, cu_dev, 0, total, plan.k, sm_scale, O, lse, stream=stream)
+        return
+    if max((b - a for a, b in zip(cu, cu[1:])), default=0) > plan.L:
+        raise DSAError("a sequence is longer than the plan")
     for s0, s1 in zip(cu, cu[1:]):
         n_tok = s1 - s0
         if n_tok == 0:
@@ -332,14 +383,10 @@ def prefill_forward_packed(plan: PrefillPlan, cu_seqlens, q8, sq, w, k8, sk, Q, 
         sl = slice(s0, s1)
         for r0 in range(0, n_tok, plan.chunk_rows):
             n = min(plan.chunk_rows, n_tok - r0)
-            if plan.fused:
-                indexer_topk(q8[sl], sq[sl], w[sl], k8[sl], sk[sl], r0, n, plan.k, plan.idx[r0:r0 + n], plan.ws,
-                             stream=stream)
-            else:
-                indexer_scores(q8[sl], sq[sl], w[sl], k8[sl], sk[sl], r0, n, plan.scores[:n],
-                               row_stats=plan.row_stats, stream=stream)
-                topk(plan.scores[:n], r0, n, plan.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws,
-                     row_stats=plan.row_stats, stream=stream)
+            indexer_scores(q8[sl], sq[sl], w[sl], k8[sl], sk[sl], r0, n, plan.scores[:n], row_stats=plan.row_stats,
+                           stream=stream)
+            topk(plan.scores[:n], r0, n, plan.k, plan.idx[r0:r0 + n], max_len=r0 + n, ws=plan.ws,
+                 row_stats=plan.row_stats, stream=stream)
         sparse_gqa_prefill(Q[sl], K[sl], V[sl], plan.idx[:n_tok], 0, n_tok, plan.k, sm_scale, O[sl],
                            None if lse is None else lse[sl], stream=stream)
         if idx_out is not None:

@@ -133,11 +133,16 @@ def test_copies_in_16_byte_pieces_need_aligned_pointers(lib):
 def test_packed_prefill_rejects_bad_offsets():
     # checked on the host before any tensor is touched
     class Plan:
-        L, D = 100, 64
+        L, D, fused = 100, 64, False
 
-    for cu in ([1, 5], [0, 5, 3], [0, 50, 200]):
-        with pytest.raises(dsa.DSAError):
-            dsa.prefill_forward_packed(Plan(), cu, *([None] * 9), None)
+    class FusedPlan(Plan):
+        fused = True
+
+    for plan in (Plan(), FusedPlan()):
+        # not starting at 0, decreasing, more tokens (or a longer sequence) than the plan holds
+        for cu in ([1, 5], [0, 5, 3], [0, 50, 200]):
+            with pytest.raises(dsa.DSAError):
+                dsa.prefill_forward_packed(plan, cu, *([None] * 9), None)
 
 
 def test_workspace_queries(lib):
