@@ -35,10 +35,12 @@ inline cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Layout of the decode workspace: [scores B x ld][idx B x k][attention partials].
+// Layout of the decode workspace: [scores B x ld][idx B x k][top-k]
+// [row key ranges 2 x B][attention split-K partials].  The key ranges are
+// preset (all-ones) at the start of each call.
 struct DecodeWs {
     int64_t ld;
-    size_t scores_off, idx_off, topk_off, attn_off, total;
+    size_t scores_off, idx_off, topk_off, range_off, attn_off, preset_bytes, total;
 };
 
 DecodeWs decode_ws_layout(int B, int max_seq_len, int Hq, int Hkv, int D, int k) {
@@ -47,7 +49,9 @@ DecodeWs decode_ws_layout(int B, int max_seq_len, int Hq, int Hkv, int D, int k)
     w.scores_off = 0;
     w.idx_off = align_up(w.scores_off + (size_t)B * w.ld * sizeof(float), 256);
     w.topk_off = align_up(w.idx_off + (size_t)B * k * sizeof(int32_t), 256);
-    w.attn_off = align_up(w.topk_off + dsa::topk_workspace_bytes(B, max_seq_len, k), 256);
+    w.range_off = align_up(w.topk_off + dsa::topk_workspace_bytes(B, max_seq_len, k), 256);
+    w.attn_off = align_up(w.range_off + (size_t)2 * B * sizeof(uint32_t), 256);
+    w.preset_bytes = (size_t)2 * B * sizeof(uint32_t);
     w.total = align_up(w.attn_off + dsa::decode_attention_workspace_bytes(B, Hq, Hkv, D, k), 256);
     return w;
 }
@@ -349,11 +353,15 @@ dsa_status_t dsa_sparse_gqa_decode(const uint16_t *q, const uint8_t *q8, const f
     float *scores = reinterpret_cast<float *>(base + L.scores_off);
     int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(base + L.idx_off);
     cudaStream_t s = as_stream(stream);
-    cudaError_t e = dsa::launch_indexer_decode(q8, q_scale, w, k8_cache, k_scale_cache, block_table, max_pages,
-                                               num_pages, seq_lens, max_seq_len, B, HI, dI, scores, L.ld, s);
+    uint32_t *keyrange = reinterpret_cast<uint32_t *>(base + L.range_off);
+    cudaError_t e = cudaMemsetAsync(keyrange, 0xFF, L.preset_bytes, s);  // row key ranges
+    if (e != cudaSuccess) return cuda_status(e);
+    bool have_range = false;
+    e = dsa::launch_indexer_decode(q8, q_scale, w, k8_cache, k_scale_cache, block_table, max_pages, num_pages,
+                                   seq_lens, max_seq_len, B, HI, dI, scores, L.ld, s, keyrange, &have_range);
     if (e != cudaSuccess) return cuda_status(e);
     e = dsa::launch_topk(scores, L.ld, 0, B, seq_lens, max_seq_len, k, idx, nullptr, base + L.topk_off,
-                         dsa::topk_workspace_bytes(B, max_seq_len, k), s);
+                         dsa::topk_workspace_bytes(B, max_seq_len, k), s, have_range ? keyrange : nullptr);
     if (e != cudaSuccess) return cuda_status(e);
     e = dsa::launch_sparse_decode(q, k_cache, v_cache, block_table, max_pages, num_pages, seq_lens, idx, B, Hq, Hkv,
                                   D, k, sm_scale, base + L.attn_off, L.total - L.attn_off, out, nullptr, s);

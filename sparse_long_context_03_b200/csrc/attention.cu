@@ -412,7 +412,7 @@ cudaError_t launch_sparse_prefill(const uint16_t *Q, const uint16_t *K, const ui
     const bool ok = dispatch_d(D, [&](auto dc) {
         constexpr int DD = decltype(dc)::value;
         constexpr int smem = kWarpsPerCta * warp_smem_bytes<DD>();
-        err = cudaFuncSetAttribute(sparse_prefill_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        err = set_smem_at_least<sparse_prefill_kernel<DD>>(smem);
         if (err != cudaSuccess) return true;
         sparse_prefill_kernel<DD><<<grid, kWarpsPerCta * 32, smem, stream>>>(Q, K, V, idx, row_begin, n_rows, Hq,
                                                                              Hkv, k, sm_scale * kLog2e, O, lse,
@@ -443,8 +443,7 @@ cudaError_t launch_sparse_decode(const uint16_t *q, const uint16_t *k_cache, con
     const bool ok = dispatch_d(D, [&](auto dc) {
         constexpr int DD = decltype(dc)::value;
         constexpr int smem = kWarpsPerCta * warp_smem_bytes<DD>();
-        err = cudaFuncSetAttribute(sparse_decode_split_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   smem);
+        err = set_smem_at_least<sparse_decode_split_kernel<DD>>(smem);
         if (err != cudaSuccess) return true;
         sparse_decode_split_kernel<DD><<<grid, kWarpsPerCta * 32, smem, stream>>>(
             q, k_cache, v_cache, block_table, max_pages, num_pages, seq_lens, idx, B, Hq, Hkv, k, s.chunk, s.nsplit,

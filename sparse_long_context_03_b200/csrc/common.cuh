@@ -136,4 +136,24 @@ __device__ __forceinline__ uint32_t order_key(float x) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// ---------------------------------------------------------------------------
+// Host: kernel attributes
+// ---------------------------------------------------------------------------
+
+// Raises a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device, calling the runtime only when the limit set so far on that
+// device is lower (one record per kernel and device).
+template <auto kernel>
+inline cudaError_t set_smem_at_least(size_t bytes) {
+    constexpr int kMaxDev = 64;
+    static size_t done[kMaxDev];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDev && __atomic_load_n(&done[dev], __ATOMIC_ACQUIRE) >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < kMaxDev) __atomic_store_n(&done[dev], bytes, __ATOMIC_RELEASE);
+    return e;
+}
+
 }  // namespace dsa

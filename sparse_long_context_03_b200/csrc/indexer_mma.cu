@@ -322,21 +322,23 @@ cudaError_t launch_indexer_prefill_mma(const uint8_t *q8, const float *sq, const
 cudaError_t launch_indexer_decode(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8c,
                                   const float *skc, const int32_t *block_table, int max_pages, int num_pages,
                                   const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI, float *scores,
-                                  int64_t ld, cudaStream_t stream) {
+                                  int64_t ld, cudaStream_t stream, uint32_t *keyrange, bool *range_written) {
+    if (range_written != nullptr) *range_written = false;
     if (B == 0 || max_seq_len == 0) return cudaSuccess;
     // the tensor-core path, unless the batch outgrows its shared-memory prefix
     // or the cache its 32-bit TMA row coordinates
-    if ((int64_t)num_pages * kPage < (1ll << 31) && indexer_decode_tc_supported(HI, dI, B, max_seq_len))
+    if ((int64_t)num_pages * kPage < (1ll << 31) && indexer_decode_tc_supported(HI, dI, B, max_seq_len)) {
+        if (range_written != nullptr) *range_written = keyrange != nullptr;
         return launch_indexer_decode_tc(q8, sq, w, k8c, skc, block_table, max_pages, num_pages, seq_lens, max_seq_len,
-                                        B, HI, dI, scores, ld, stream);
+                                        B, HI, dI, scores, ld, keyrange, stream);
+    }
     const int pages = (max_seq_len + kPage - 1) / kPage;
     const dim3 grid((pages + kDecodePagesPerCta - 1) / kDecodePagesPerCta, B);
     cudaError_t err = cudaSuccess;
     const bool ok = dispatch_shape(HI, dI, [&](auto di, auto nt) {
         constexpr int DI = decltype(di)::value, NT = decltype(nt)::value;
         constexpr int smem = kDecodeWarps * 2 * page_stage_bytes<DI>();
-        err = cudaFuncSetAttribute(indexer_decode_mma_kernel<DI, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   smem);
+        err = set_smem_at_least<indexer_decode_mma_kernel<DI, NT>>(smem);
         if (err != cudaSuccess) return true;
         indexer_decode_mma_kernel<DI, NT><<<grid, kDecodeWarps * 32, smem, stream>>>(
             q8, sq, w, k8c, skc, block_table, max_pages, num_pages, seq_lens, max_seq_len, HI, scores, ld);

@@ -565,7 +565,7 @@ __global__ void __maxnreg__(kDecMaxRegs) indexer_decode_tc_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const uint8_t *__restrict__ q8, const float *__restrict__ sq,
     const float *__restrict__ w, const float *__restrict__ skc, const int32_t *__restrict__ block_table,
     int max_pages, int num_pages, const int32_t *__restrict__ seq_lens, int max_seq_len, int B, int HI,
-    float *__restrict__ scores, int64_t ld) {
+    float *__restrict__ scores, int64_t ld, uint32_t *__restrict__ keyrange) {
     using Lay = DecLayout<N, DI>;
     constexpr int S = Lay::kStages, A = Lay::kAccBufs, G = kDecGroups;
     constexpr int SP = Lay::SP, T = Lay::kTiles, PPW = SP / kDecProducers;  // pages per producer warp
@@ -800,6 +800,26 @@ __global__ void __maxnreg__(kDecMaxRegs) indexer_decode_tc_kernel(
         int cur_b = -1;
         float wv[N];
         float sqb = 0.f;
+        // Each row's score range for the top-k, as order keys:
+        // keyrange[b] = min key, keyrange[B + b] = complement of the max key
+        // (both preset to all-ones, so atomicMin keeps each).  A warp keeps a
+        // running range over its consecutive steps of one sequence and adds
+        // it in when the sequence changes and at the end.
+        int rng_b = -1;
+        float rng_lo = INFINITY, rng_hi = -INFINITY;
+        auto flush_range = [&]() {
+            if (keyrange == nullptr || rng_b < 0) return;
+            const uint32_t klo =
+                __reduce_min_sync(0xFFFFFFFFu, rng_lo == INFINITY ? 0xFFFFFFFFu : order_key(rng_lo));
+            const uint32_t khi =
+                __reduce_min_sync(0xFFFFFFFFu, rng_hi == -INFINITY ? 0xFFFFFFFFu : ~order_key(rng_hi));
+            if (lane == 0 && rng_b < B) {
+                atomicMin(keyrange + rng_b, klo);
+                atomicMin(keyrange + B + rng_b, khi);
+            }
+            rng_lo = INFINITY;
+            rng_hi = -INFINITY;
+        };
 #pragma unroll
         for (int h = 0; h < N; ++h) wv[h] = 0.f;
         bool ok = true;
@@ -845,14 +865,23 @@ __global__ void __maxnreg__(kDecMaxRegs) indexer_decode_tc_kernel(
                 tc::mbar_arrive(tempty_bar(a));
                 tc::mbar_arrive(empty_bar(s));
             }
+            if (keyrange != nullptr && meta.x != rng_b) {
+                flush_range();
+                rng_b = meta.x;
+            }
 #pragma unroll
             for (int t = 0; t < T; ++t) {
                 const int pi = 2 * t + (qw >> 1);  // page of the step
                 const int tok = (SP * meta.y + pi) * kDecPage + (qw & 1) * 32 + lane;
-                if (tok < meta.z)
-                    scores[(size_t)cur_b * ld + tok] = ((meta.w >> pi) & 1) ? v[t] * sqb * sk[t] : -INFINITY;
+                if (tok < meta.z) {
+                    const float sc = ((meta.w >> pi) & 1) ? v[t] * sqb * sk[t] : -INFINITY;
+                    scores[(size_t)cur_b * ld + tok] = sc;
+                    rng_lo = fminf(rng_lo, sc);
+                    rng_hi = fmaxf(rng_hi, sc);
+                }
             }
         }
+        if (ok) flush_range();
         if (!ok) record_timeout();
     }
 
@@ -901,22 +930,6 @@ int sm_count() {
     return n > 0 ? n : 148;
 }
 
-// Sets a kernel's dynamic shared-memory limit once per device (the
-// attribute is per device and does not change).  One instantiation, and so
-// one set of flags, per kernel.
-template <auto kernel>
-cudaError_t set_smem_once(int smem) {
-    constexpr int kMaxDev = 64;
-    static int done[kMaxDev];
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDev && __atomic_load_n(&done[dev], __ATOMIC_ACQUIRE)) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess && dev >= 0 && dev < kMaxDev) __atomic_store_n(&done[dev], 1, __ATOMIC_RELEASE);
-    return e;
-}
-
 template <int HI, int DI, int MODE, bool VARLEN>
 cudaError_t launch_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8, const float *sk, int L,
                       int row_begin, int n_rows, const EpiArgs &a, cudaStream_t stream) {
@@ -930,7 +943,7 @@ cudaError_t launch_tc(const uint8_t *q8, const float *sq, const float *w, const 
     const int grid = nb < sm_count() ? nb : sm_count();
     // at least 116 KB so that one CTA (and its 512 TMEM columns) owns each SM
     constexpr int smem = Layout<DI>::kAlloc > 116 * 1024 ? Layout<DI>::kAlloc : 116 * 1024;
-    cudaError_t e = set_smem_once<indexer_tc_kernel<HI, DI, MODE, VARLEN>>(smem);
+    cudaError_t e = set_smem_at_least<indexer_tc_kernel<HI, DI, MODE, VARLEN>>(smem);
     if (e != cudaSuccess) return e;
     indexer_tc_kernel<HI, DI, MODE, VARLEN><<<grid, EpiShape<HI>::kThreads, smem, stream>>>(mk, mq, sq, w, sk,
                                                                                            row_begin, n_rows, a);
@@ -940,15 +953,15 @@ cudaError_t launch_tc(const uint8_t *q8, const float *sq, const float *w, const 
 template <int N, int DI>
 cudaError_t launch_decode_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8c, const float *skc,
                              const int32_t *block_table, int max_pages, int num_pages, const int32_t *seq_lens,
-                             int max_seq_len, int B, int HI, float *scores, int64_t ld, cudaStream_t stream) {
+                             int max_seq_len, int B, int HI, float *scores, int64_t ld, uint32_t *keyrange,
+                             cudaStream_t stream) {
     CUtensorMap mk;
     if (!make_map(&mk, k8c, (uint64_t)num_pages * kDecPage, DI, kDecPage)) return cudaErrorInvalidValue;
     constexpr int smem = DecLayout<N, DI>::kAlloc > 116 * 1024 ? DecLayout<N, DI>::kAlloc : 116 * 1024;
-    cudaError_t e =
-        cudaFuncSetAttribute(indexer_decode_tc_kernel<N, DI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_smem_at_least<indexer_decode_tc_kernel<N, DI>>(smem);
     if (e != cudaSuccess) return e;
     indexer_decode_tc_kernel<N, DI><<<sm_count(), kDecThreads, smem, stream>>>(
-        mk, q8, sq, w, skc, block_table, max_pages, num_pages, seq_lens, max_seq_len, B, HI, scores, ld);
+        mk, q8, sq, w, skc, block_table, max_pages, num_pages, seq_lens, max_seq_len, B, HI, scores, ld, keyrange);
     return cudaGetLastError();
 }
 
@@ -1058,17 +1071,17 @@ bool indexer_decode_tc_supported(int HI, int dI, int B, int max_seq_len) {
 cudaError_t launch_indexer_decode_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8c,
                                      const float *skc, const int32_t *block_table, int max_pages, int num_pages,
                                      const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI, float *scores,
-                                     int64_t ld, cudaStream_t stream) {
+                                     int64_t ld, uint32_t *keyrange, cudaStream_t stream) {
     if (B == 0 || max_seq_len == 0) return cudaSuccess;
     auto by_di = [&](auto n) -> cudaError_t {
         constexpr int NN = decltype(n)::value;
         switch (dI) {
             case 32: return launch_decode_tc<NN, 32>(q8, sq, w, k8c, skc, block_table, max_pages, num_pages, seq_lens,
-                                                     max_seq_len, B, HI, scores, ld, stream);
+                                                     max_seq_len, B, HI, scores, ld, keyrange, stream);
             case 64: return launch_decode_tc<NN, 64>(q8, sq, w, k8c, skc, block_table, max_pages, num_pages, seq_lens,
-                                                     max_seq_len, B, HI, scores, ld, stream);
+                                                     max_seq_len, B, HI, scores, ld, keyrange, stream);
             case 128: return launch_decode_tc<NN, 128>(q8, sq, w, k8c, skc, block_table, max_pages, num_pages,
-                                                       seq_lens, max_seq_len, B, HI, scores, ld, stream);
+                                                       seq_lens, max_seq_len, B, HI, scores, ld, keyrange, stream);
             default: return cudaErrorInvalidValue;
         }
     };

@@ -14,10 +14,14 @@ cudaError_t launch_indexer_prefill_mma(const uint8_t *q8, const float *sq, const
                                        int64_t ld, cudaStream_t stream);
 cudaError_t launch_row_stats(const float *scores, int64_t ld, int row_begin, int n_rows, float *row_stats,
                              cudaStream_t stream);
+// keyrange (optional, [2, B] uint32, every word preset to all-ones): the
+// tensor-core path records each row's (min order key, complemented max
+// order key) there and sets *range_written.
 cudaError_t launch_indexer_decode(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8c,
                                   const float *skc, const int32_t *block_table, int max_pages, int num_pages,
                                   const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI, float *scores,
-                                  int64_t ld, cudaStream_t stream);
+                                  int64_t ld, cudaStream_t stream, uint32_t *keyrange = nullptr,
+                                  bool *range_written = nullptr);
 
 // indexer_tc.cu
 bool indexer_tc_supported(int HI, int dI);
@@ -46,14 +50,17 @@ bool indexer_decode_tc_supported(int HI, int dI, int B, int max_seq_len);
 cudaError_t launch_indexer_decode_tc(const uint8_t *q8, const float *sq, const float *w, const uint8_t *k8c,
                                      const float *skc, const int32_t *block_table, int max_pages, int num_pages,
                                      const int32_t *seq_lens, int max_seq_len, int B, int HI, int dI, float *scores,
-                                     int64_t ld, cudaStream_t stream);
+                                     int64_t ld, uint32_t *keyrange, cudaStream_t stream);
 
 // topk.cu
 size_t topk_workspace_bytes(int n_rows, int max_len, int k);
 bool topk_k_supported(int k);
+// row_keyrange (optional, [2, n_rows] as written by the decode indexer):
+// each row's score range, used by the few-long-rows path in place of its
+// range pass
 cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_rows, const int32_t *row_len,
                         int max_len, int k, int32_t *idx, const float *row_stats, void *ws, size_t ws_bytes,
-                        cudaStream_t stream);
+                        cudaStream_t stream, const uint32_t *row_keyrange = nullptr);
 
 // topk_fused.cu: the fused indexer + top-k (sampled threshold, candidate
 // indexer, exact selection of the candidates, repair of undecided rows)

@@ -621,7 +621,8 @@ __host__ __device__ constexpr size_t cluster_smem_bytes(int k) { return smem_byt
 __global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads)
     topk_rows_cluster_kernel(const float *__restrict__ scores, int64_t ld, int row_begin,
                              const int32_t *__restrict__ row_len, int max_len, int k, int32_t *__restrict__ idx,
-                             const float *__restrict__ row_stats) {
+                             const float *__restrict__ row_stats, const uint32_t *__restrict__ row_keyrange,
+                             int n_rows) {
     namespace cgs = cooperative_groups;
     cgs::cluster_group cluster = cgs::this_cluster();
     const int rank = (int)cluster.block_rank();
@@ -651,6 +652,12 @@ __global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads)
         if (tid < 4) {
             vmin = __ldg(row_stats + (size_t)r * 8 + 2 * tid);
             vmax = __ldg(row_stats + (size_t)r * 8 + 2 * tid + 1);
+        }
+    } else if (row_keyrange != nullptr) {
+        // the decode indexer's record: min order key, complemented max key
+        if (tid == 0) {
+            vmin = key_value(__ldg(row_keyrange + r));
+            vmax = key_value(~__ldg(row_keyrange + n_rows + r));
         }
     } else {
         for (int i0 = tid * kVec; i0 < m; i0 += kChunk) {
@@ -800,7 +807,7 @@ size_t topk_workspace_bytes(int, int, int) { return 0; }
 
 cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_rows, const int32_t *row_len,
                         int max_len, int k, int32_t *idx, const float *row_stats, void *, size_t,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, const uint32_t *row_keyrange) {
     if (n_rows == 0) return cudaSuccess;
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
@@ -809,17 +816,15 @@ cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_ro
         // few long rows: a cluster of CTAs per row keeps every SM busy
         const size_t csmem = cluster_smem_bytes(k);
         if (csmem > 220 * 1024) return cudaErrorInvalidValue;
-        cudaError_t e = cudaFuncSetAttribute(topk_rows_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)csmem);
+        cudaError_t e = set_smem_at_least<topk_rows_cluster_kernel>(csmem);
         if (e != cudaSuccess) return e;
-        topk_rows_cluster_kernel<<<n_rows * kClusterSize, kThreads, csmem, stream>>>(scores, ld, row_begin, row_len,
-                                                                                       max_len, k, idx, row_stats);
+        topk_rows_cluster_kernel<<<n_rows * kClusterSize, kThreads, csmem, stream>>>(
+            scores, ld, row_begin, row_len, max_len, k, idx, row_stats, row_keyrange, n_rows);
         return cudaGetLastError();
     }
     if (bitmap_smem_bytes(max_len) <= (size_t)kBitmapSmemMax) {
         const size_t bsmem = bitmap_smem_bytes(max_len);
-        cudaError_t e = cudaFuncSetAttribute(topk_rows_bitmap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)bsmem);
+        cudaError_t e = set_smem_at_least<topk_rows_bitmap_kernel>(bsmem);
         if (e != cudaSuccess) return e;
         topk_rows_bitmap_kernel<<<n_rows, kThreads, bsmem, stream>>>(scores, ld, row_begin, row_len, max_len, k, idx,
                                                                      row_stats);
@@ -827,7 +832,7 @@ cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_ro
     }
     const size_t smem = smem_bytes(k);
     if (smem > 220 * 1024) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem_at_least<topk_rows_kernel>(smem);
     if (e != cudaSuccess) return e;
     topk_rows_kernel<<<n_rows, kThreads, smem, stream>>>(scores, ld, row_begin, row_len, max_len, k, idx,
                                                          row_stats);

@@ -523,21 +523,6 @@ int sm_count_here() {
     return n > 0 ? n : 148;
 }
 
-// Raises a kernel's dynamic shared-memory limit to `bytes` when it is lower
-// (once per device and size; one instantiation, and so one set of
-// records, per kernel).
-template <auto kernel>
-cudaError_t set_smem(size_t bytes) {
-    constexpr int kMaxDev = 64;
-    static size_t done[kMaxDev];
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDev && __atomic_load_n(&done[dev], __ATOMIC_ACQUIRE) >= bytes) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e == cudaSuccess && dev >= 0 && dev < kMaxDev) __atomic_store_n(&done[dev], bytes, __ATOMIC_RELEASE);
-    return e;
-}
 
 }  // namespace
 
@@ -620,7 +605,7 @@ cudaError_t launch_indexer_topk_stage(int stage, const uint8_t *q8, const float 
             if (e != cudaSuccess) return e;
         }
         // thresholds (and the repair list emptied)
-        e = set_smem<sample_threshold_kernel>(sizeof(ThreshSmem));
+        e = set_smem_at_least<sample_threshold_kernel>(sizeof(ThreshSmem));
         if (e != cudaSuccess) return e;
         sample_threshold_kernel<<<n_rows, kThreads, sizeof(ThreshSmem), stream>>>(
             P.sample, lay.lds, row_begin, n_rows, k, lay.keep_all, indexer_sample_stride(), P.tau, P.repair,
@@ -638,12 +623,12 @@ cudaError_t launch_indexer_topk_stage(int stage, const uint8_t *q8, const float 
     if (stage == 3) {
         // exact selection, then the repair of the listed rows (which exits at
         // once when there are none)
-        e = set_smem<cand_select_kernel>(lay.select_smem);
+        e = set_smem_at_least<cand_select_kernel>(lay.select_smem);
         if (e != cudaSuccess) return e;
         cand_select_kernel<<<n_rows, kThreads, lay.select_smem, stream>>>(P.cand, P.counts, lay.seg_cap, row_begin,
                                                                           k, idx, P.repair, P.cand_total, cu, nseq);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        e = set_smem<repair_rows_kernel>(lay.repair_smem);
+        e = set_smem_at_least<repair_rows_kernel>(lay.repair_smem);
         if (e != cudaSuccess) return e;
         repair_rows_kernel<<<lay.repair_ctas, kRepairThreads, lay.repair_smem, stream>>>(
             q8, sq, w, k8, sk, HI, dI, row_begin, k, P.repair, P.scratch, lay.scratch_ld, idx, cu, nseq);
