@@ -61,6 +61,21 @@ def test_indexer_exact_inputs_bit_exact(HI, dI, L):
     assert np.array_equal(got[:, :L][tri].astype(np.float64), ref[tri])
 
 
+def test_indexer_exact_inputs_bit_exact_8k_many_blocks_per_cta():
+    # L = 8192 in one launch: 2048 query blocks over the persistent CTAs
+    # (about 14 each) and up to 32 key steps per block, so the 8-stage key
+    # ring wraps many times within and across blocks
+    L, HI, dI = 8192, 32, 64
+    d = inputs.exact_indexer_inputs(L, HI, dI, seed=808)
+    got = gpu_scores(_gpu(d), 0, L, L)
+    h = {k: H(d[k]) for k in ("q8", "sq", "w", "k8", "sk")}
+    rng = np.random.default_rng(8)
+    rows = sorted({0, 3, 255, 256, 511, 4095, 4096, 6000, L - 5, L - 1} | set(int(x) for x in rng.integers(0, L, 8)))
+    for t in rows:
+        ref = oracle.indexer(h["q8"], h["sq"], h["w"], h["k8"], h["sk"], row_begin=t, n_rows=1)[0]
+        assert np.array_equal(got[t, : t + 1], ref[: t + 1]), f"row {t}"
+
+
 def test_indexer_signed_weights():
     cfg = inputs.config(0)
     d = inputs.prefill_inputs(cfg, L=300, seed=44)
@@ -466,6 +481,19 @@ def check_decode(cfg, dh, out, idx, k):
                                       ref_idx, cfg.sm_scale)
     same = np.all(idx == ref_idx, axis=1)
     check_attention(out[same], Oref[same], what="decode")
+    if not same.all():
+        # sequences whose set differs from the oracle's by near-ties: the
+        # attention stage alone on the oracle's sets, so every sequence's
+        # output is checked
+        g = {kk: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for kk, v in dh.items()}
+        B = len(h["seq_lens"])
+        ws = torch.empty(dsa.decode_attention_workspace_size(B, cfg.Hq, cfg.Hkv, cfg.D, k), dtype=torch.uint8,
+                         device=DEV)
+        o3 = torch.empty(B, cfg.Hq, cfg.D, dtype=torch.bfloat16, device=DEV)
+        dsa.sparse_gqa_decode_attention(g["q"], g["k_cache"], g["v_cache"], g["block_table"], g["seq_lens"],
+                                        torch.from_numpy(ref_idx).to(DEV), k, cfg.sm_scale, ws, o3)
+        torch.cuda.synchronize()
+        check_attention(o3.float().cpu().numpy()[~same], Oref[~same], what="decode (oracle index sets)")
     return I, ref_idx, Oref
 
 
