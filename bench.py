@@ -285,7 +285,7 @@ class PrefillBench:
     def flops_threshold(self, r0, n):
         """The sampled scores: every 32nd key of the rows scored from candidates."""
         c = self.cfg
-        keep_all = max(8192, 2 * c.k + 2048)
+        keep_all = 4 * max(3 * c.k // 4, 1024)  # rows with more keys than this are sampled
         lo = max(r0, keep_all)
         return 2 * c.HI * c.dI * sum(t // 32 + 1 for t in range(lo, r0 + n))
 

@@ -13,7 +13,7 @@
 //      (1/32 of the work);
 //   2. sample_threshold_kernel: tau_t = (just below) the r-th largest sampled
 //      score of row t, where r is the expected number of sampled keys among
-//      the row's k winners plus seven standard deviations plus eight -- so
+//      the row's k winners plus six standard deviations plus eight -- so
 //      that, with overwhelming probability, at least k scores of the row are
 //      >= tau_t and at most a few thousand are.  Rows with at most keep_all
 //      visible keys get tau = -inf (every key is a candidate);
@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kThreads) sample_threshold_kernel(const float 
     }
     const int m = t / stride - (start + stride - 1) / stride + 1;  // sampled keys visible to row t
     const float mu = (float)k * (float)m / (float)n;
-    const int rsel = (int)ceilf(mu + 7.f * sqrtf(mu) + 8.f);
+    const int rsel = (int)ceilf(mu + 6.f * sqrtf(mu) + 8.f);
     if (rsel >= m) {
         if (tid == 0) tau[r] = -INFINITY;
         return;
@@ -168,14 +168,16 @@ struct SelectSmem {
 // lists instead.
 constexpr int kBitmapMaxN = 262144;
 
-__host__ __device__ constexpr size_t select_tail_bytes(int seg_cap, int k) {
-    return (size_t)kBitmapMaxN / 8 > (size_t)kSegs * seg_cap + (size_t)k * 4 + 16
-               ? (size_t)kBitmapMaxN / 8
-               : (size_t)kSegs * seg_cap + (size_t)k * 4 + 16;
+// The tail holds the bitmap of the chunk's longest row (up to kBitmapMaxN
+// keys) or, for longer rows, the merge path's flags and lists.
+__host__ __device__ constexpr size_t select_tail_bytes(int seg_cap, int k, int max_n) {
+    const size_t bitmap = ((size_t)(max_n < kBitmapMaxN ? max_n : kBitmapMaxN) + 127) / 128 * 16;
+    const size_t merge = max_n > kBitmapMaxN ? (size_t)kSegs * seg_cap + (size_t)k * 4 + 16 : 0;
+    return bitmap > merge ? bitmap : merge;
 }
 
-__host__ __device__ constexpr size_t select_smem_bytes(int seg_cap, int k) {
-    return (sizeof(SelectSmem) + 15) / 16 * 16 + (size_t)kSegs * seg_cap * 8 + select_tail_bytes(seg_cap, k);
+__host__ __device__ constexpr size_t select_smem_bytes(int seg_cap, int k, int max_n) {
+    return (sizeof(SelectSmem) + 15) / 16 * 16 + (size_t)kSegs * seg_cap * 8 + select_tail_bytes(seg_cap, k, max_n);
 }
 
 __device__ __forceinline__ void flag_repair(int *repair, int r) {
@@ -531,8 +533,11 @@ FusedTopkLayout fused_topk_layout(int row_begin, int n_rows, int k, int HI, int 
     const int row_end = row_begin + n_rows;
     const int stride = indexer_sample_stride();
     // candidates per row: room for about twice what the threshold lets through
-    L.keep_all = k * 2 + 2048 > 8192 ? k * 2 + 2048 : 8192;
-    L.seg_cap = L.keep_all / kSegs + 32;  // a row with keep_all keys fits (each quarter <= n/4 + 32)
+    // a segment holds about twice its share of what the threshold lets
+    // through (about k + 6 sqrt(32 k) + 256 per row); a row with at most
+    // keep_all keys keeps them all (each quarter holds at most n/4 + 32)
+    L.seg_cap = (3 * k / 4 > 1024 ? 3 * k / 4 : 1024) + 32;
+    L.keep_all = kSegs * (L.seg_cap - 32);
     L.lds = ((row_end > 0 ? (row_end - 1) / stride + 1 : 1) + 3) / 4 * 4;
     L.repair_ctas = sm_count_here();
     L.scratch_ld = ((row_end > 0 ? row_end : 1) + 3) / 4 * 4;
@@ -552,14 +557,15 @@ FusedTopkLayout fused_topk_layout(int row_begin, int n_rows, int k, int HI, int 
     L.scratch_off = off;
     off = align256(off + (size_t)L.repair_ctas * L.scratch_ld * 4);
     L.total = off;
-    L.select_smem = select_smem_bytes(L.seg_cap, k);
+    L.select_smem = select_smem_bytes(L.seg_cap, k, row_end > 0 ? row_end : 1);
     L.repair_smem = (sizeof(TopkSmem) + 15) / 16 * 16 + ((size_t)HI * dI + HI) * 4;
     return L;
 }
 
 bool fused_topk_supported(int k, int HI, int dI) {
     if (k < 1 || !indexer_tc_supported(HI, dI)) return false;
-    const FusedTopkLayout L = fused_topk_layout(0, 1, k, HI, dI);
+    // the worst case is a chunk whose rows take the merge path
+    const FusedTopkLayout L = fused_topk_layout(0, kBitmapMaxN + 1, k, HI, dI);
     return L.select_smem <= 200 * 1024 && L.repair_smem <= 200 * 1024;
 }
 

@@ -4,8 +4,8 @@ unfused path (dsa_indexer_scores + dsa_topk).
 
 What must hold (criteria of parity_helpers): bit-exact Omega_t on
 exact-arithmetic inputs, whichever way a row is decided -- from the
-candidates at or above its sampled threshold (rows with more than 8192
-visible keys), from all of its keys (shorter rows), or by the full re-scoring
+candidates at or above its sampled threshold (rows with more than 6144
+visible keys at k = 2048), from all of its keys (shorter rows), or by the full re-scoring
 of a row the candidates cannot decide (massive exact ties); on random inputs
 the near-tie criterion, and the same indices as the unfused path, which
 computes the same fp32 scores.
@@ -21,7 +21,7 @@ from sparse_long_context_03_b200 import dsa, inputs
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
-KEEP_ALL = 8192  # rows with at most this many keys keep every key as a candidate (k <= 3072)
+KEEP_ALL = 6144  # rows with at most this many keys keep every key as a candidate (k = 2048)
 
 
 def H(t):
