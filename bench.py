@@ -780,6 +780,51 @@ def stage_roofline(per, pb, pk, src, fp8, reads):
     return out
 
 
+# ----------------------------------------------------------------------------
+# untimed cases for profiler captures (no JSON bench line)
+# ----------------------------------------------------------------------------
+
+def omega_union(plan, L, k, width=16, fracs=(0.125, 0.25, 0.5, 0.75, 0.99), samples=32):
+    """Distinct key positions selected by `width` adjacent queries (the Top-KV
+    dedup's potential), at `samples` starting rows near each fraction of L."""
+    res = {}
+    for frac in fracs:
+        sizes = []
+        for j in range(samples):
+            t0 = min(int(L * frac) + 4096 * j, L - width) // width * width
+            blk = plan.idx[t0:t0 + width].flatten()
+            sizes.append(int(torch.unique(blk[blk >= 0]).numel()))
+        res[f"t~{int(L * frac)}"] = {"mean_union": sum(sizes) / len(sizes), "min": min(sizes), "max": max(sizes),
+                                     "of_width_k": sum(sizes) / len(sizes) / (width * k)}
+    return res
+
+
+def run_profile_case(args):
+    """One GPU, no timing: `fused` runs the fused indexer + top-k of the
+    workload twice, `attention` selects once and runs the prefill attention
+    twice (the second launch of each is the one to capture); `omega-union`
+    prints the union of Omega over 16 adjacent queries as JSON."""
+    from sparse_long_context_03_b200 import build, dsa, inputs
+    build.build()
+    cfg = inputs.config(args.config)
+    d = inputs.prefill_inputs(cfg, device="cuda")
+    plan = dsa.PrefillPlan(cfg.L, cfg.HI, cfg.dI, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, chunk_rows=args.chunk_rows,
+                           device="cuda", fused=False if args.unfused else True)
+    case = args.profile_case
+    for _ in range(2 if case == "fused" else 1):
+        dsa.select_rows(plan, d["q8"], d["sq"], d["w"], d["k8"], d["sk"])
+    if case == "attention":
+        O = torch.empty(cfg.L, cfg.Hq, cfg.D, dtype=torch.bfloat16, device="cuda")
+        for _ in range(2):
+            dsa.sparse_gqa_prefill(d["Q"], d["K"], d["V"], plan.idx, 0, cfg.L, cfg.k, cfg.sm_scale, O)
+    torch.cuda.synchronize()
+    if case == "omega-union":
+        print(json.dumps({"workload": cfg.name, "omega_union_16": omega_union(plan, cfg.L, cfg.k)}))
+    else:
+        print(json.dumps({"workload": cfg.name, "profile_case": case, "status": "ok"}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -798,8 +843,12 @@ def main():
                     help="materialise the score matrix per chunk and run dsa_topk (instead of dsa_indexer_topk)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="sequences in the decode workload (default: the decode-b32 layer's 32)")
+    ap.add_argument("--profile-case", default=None, choices=["fused", "attention", "omega-union"],
+                    help="run one untimed case on one GPU for a profiler capture (no bench line)")
     args = ap.parse_args()
 
+    if args.profile_case is not None:
+        return run_profile_case(args)
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         world = int(os.environ.get("WORLD_SIZE", "1"))
