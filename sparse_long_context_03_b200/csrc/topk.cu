@@ -599,13 +599,23 @@ __global__ void __launch_bounds__(kThreads) topk_rows_bitmap_kernel(const float 
 // Long rows, few of them (decode): one thread-block cluster per row.
 //
 // The row is cut into kClusterSize contiguous slices, one per CTA.  Each pass
-// runs on every slice in parallel; the row's value range, the bucket
-// histogram and the per-slice winner / candidate lists are combined through
-// distributed shared memory.  Every exchange is bracketed by hardware cluster
-// barriers (no flag polling), and a CTA leaves only after the last barrier
-// that follows any remote read of its shared memory.  Rank 0 gathers the
-// lists -- slices are in index order, so concatenation keeps the lists
-// ascending -- and finishes the row exactly as the single-CTA kernel does.
+// runs on every slice in parallel; the row's value range (unless the indexer
+// recorded it) and the bucket histogram are combined through distributed
+// shared memory.  Every exchange is bracketed by hardware cluster barriers
+// (no flag polling), and a CTA leaves only after the last barrier that
+// follows any remote access to its shared memory.
+//
+// Usual case (at most kSmallCand entries in the threshold bucket, slices of
+// at most 32k entries): every CTA reads each slice's winner and candidate
+// counts from the other CTAs' histograms, marks its own winners in a bitmap
+// of its slice, and writes its candidates into every CTA's candidate list
+// at its slice's offset.  After one barrier every CTA ranks all candidates
+// (larger key first, then lower index), marks the chosen ones of its slice
+// and writes its slice's set bits in ascending order at its slice's output
+// offset -- the output is written by all CTAs at once.  Otherwise rank 0
+// gathers the per-slice ordered lists (slices are in index order, so
+// concatenation keeps them ascending) and finishes the row as the single-CTA
+// kernel does.
 // ---------------------------------------------------------------------------
 
 constexpr int kClusterSize = 8;
@@ -614,11 +624,17 @@ struct ClusterExtra {
     uint32_t ghist[kNB];   // the row's histogram (sum over the cluster)
     float range[2];        // this slice's min, max
     uint32_t counts[2];    // this slice's winners, candidates
+    // usual case: per slice, entries above the threshold bucket, entries in
+    // it, and chosen candidates; this slice's candidates written so far
+    uint32_t slice_above[kClusterSize];
+    uint32_t slice_cand[kClusterSize];
+    uint32_t slice_chosen[kClusterSize];
+    uint32_t ncand;
 };
 
 __host__ __device__ constexpr size_t cluster_smem_bytes(int k) { return smem_bytes(k) + sizeof(ClusterExtra); }
 
-__global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads)
+__global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads, 2)
     topk_rows_cluster_kernel(const float *__restrict__ scores, int64_t ld, int row_begin,
                              const int32_t *__restrict__ row_len, int max_len, int k, int32_t *__restrict__ idx,
                              const float *__restrict__ row_stats, const uint32_t *__restrict__ row_keyrange,
@@ -692,15 +708,22 @@ __global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads)
         cx.range[0] = a;
         cx.range[1] = b;
     }
-    cluster.sync();
-    vmin = INFINITY;
-    vmax = -INFINITY;
-    for (int q = 0; q < kClusterSize; ++q) {
-        const float *rr = cluster.map_shared_rank(cx.range, q);
-        vmin = fminf(vmin, rr[0]);
-        vmax = fmaxf(vmax, rr[1]);
+    if (row_stats != nullptr || row_keyrange != nullptr) {
+        // every CTA read the same record: nothing to exchange
+        __syncthreads();
+        vmin = cx.range[0];
+        vmax = cx.range[1];
+    } else {
+        cluster.sync();
+        vmin = INFINITY;
+        vmax = -INFINITY;
+        for (int q = 0; q < kClusterSize; ++q) {
+            const float *rr = cluster.map_shared_rank(cx.range, q);
+            vmin = fminf(vmin, rr[0]);
+            vmax = fmaxf(vmax, rr[1]);
+        }
+        cluster.sync();  // every remote read of the ranges is done
     }
-    cluster.sync();  // every remote read of the ranges is done
     if (vmin == vmax) {  // every entry ties: the k lowest indices
         if (rank == 0)
             for (int i = tid; i < k; i += kThreads) out[i] = i;
@@ -734,7 +757,89 @@ __global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads)
     const uint32_t need = sm.bcast[1];
     const uint32_t n_above = sm.bcast[2];
     const uint32_t cnt = cx.ghist[Bt];
+    uint32_t *bm = reinterpret_cast<uint32_t *>(alist);  // usual case: this slice's bitmap
+    const int bm_words = (chunk + 31) / 32;
+    const bool usual = cnt <= (uint32_t)kSmallCand && bm_words <= k;
+    if (usual) {
+        if (warp < kClusterSize) {  // warp q reads slice q's counts
+            const uint32_t *hq = cluster.map_shared_rank(sm.hist, warp);
+            uint32_t a = 0;
+            for (int b = (int)Bt + 1 + lane; b < kNB; b += 32) a += hq[b];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
+            if (lane == 0) {
+                cx.slice_above[warp] = a;
+                cx.slice_cand[warp] = hq[Bt];
+                cx.slice_chosen[warp] = 0;
+            }
+        }
+        if (tid == 0) cx.ncand = 0;
+        for (int w = tid; w < bm_words; w += kThreads) bm[w] = 0;
+        __syncthreads();
+    }
     cluster.sync();  // every remote read of the histograms is done
+    if (usual) {
+        uint32_t coff = 0;  // this slice's first slot in the row's candidate list
+        for (int q = 0; q < rank; ++q) coff += cx.slice_cand[q];
+        for (int i0 = tid * kVec; i0 < m; i0 += kChunk) {
+            float x[kVec];
+            const int c = load_vals(srow, i0, m, x);
+            uint32_t win = 0;
+#pragma unroll
+            for (int j = 0; j < kVec; ++j) {
+                if (j >= c) continue;
+                const uint32_t b = bucket_of(x[j], vmin, scale);
+                if (b > Bt) {
+                    win |= 1u << j;
+                } else if (b == Bt) {
+                    const uint32_t pos = coff + atomicAdd(&cx.ncand, 1u);
+                    const uint32_t key = order_key(x[j]);
+                    for (int q = 0; q < kClusterSize; ++q) {
+                        cluster.map_shared_rank(sm.ckey, q)[pos] = key;
+                        cluster.map_shared_rank(sm.cidx, q)[pos] = lo + i0 + j;
+                    }
+                }
+            }
+            // i0 is a multiple of kVec = 16: the group is one half of a word
+            if (win) atomicOr(&bm[i0 >> 5], win << (i0 & 31));
+        }
+        __syncthreads();
+        cluster.sync();  // every CTA holds the row's cnt candidates; no remote access follows
+
+        if (tid < (int)cnt) {
+            const uint32_t ki = sm.ckey[tid];
+            const int32_t xi = sm.cidx[tid];
+            uint32_t rk = 0;
+            for (int j = 0; j < (int)cnt; ++j) {
+                const uint32_t kj = sm.ckey[j];
+                rk += (kj > ki) || (kj == ki && sm.cidx[j] < xi);
+            }
+            if (rk < need) {
+                const int q = xi / chunk;
+                atomicAdd(&cx.slice_chosen[q], 1u);
+                if (q == rank) atomicOr(&bm[(xi - lo) >> 5], 1u << ((xi - lo) & 31));
+            }
+        }
+        __syncthreads();
+        uint32_t off = 0;  // this slice's first output position
+        for (int q = 0; q < rank; ++q) off += cx.slice_above[q] + cx.slice_chosen[q];
+        const int words = (m + 31) / 32;
+        const int per = (words + kThreads - 1) / kThreads;
+        const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
+        uint32_t mine = 0;
+        for (int w = w0; w < w1; ++w) mine += __popc(bm[w]);
+        uint32_t tot;
+        uint32_t pos = off + block_scan_packed(mine, sm.red, &tot);
+        for (int w = w0; w < w1; ++w) {
+            uint32_t v = bm[w];
+            while (v) {
+                const int b = __ffs(v) - 1;
+                v &= v - 1u;
+                out[pos++] = lo + w * 32 + b;
+            }
+        }
+        return;
+    }
     if (cnt > (uint32_t)kCap) {
         if (rank == 0) topk_row_radix(row, n, k, out, sm);
         return;

@@ -173,6 +173,40 @@ def test_topk_many_long_rows_bit_exact():
     assert np.array_equal(got, oracle.topk(x.astype(np.float64), lens, 2048))
 
 
+@pytest.mark.parametrize("k", [512, 2048])
+@pytest.mark.parametrize("stats", [False, True])
+def test_topk_cluster_rows_bit_exact(k, stats):
+    # Fewer rows than SMs and rows past 16384 entries: one 8-CTA cluster per
+    # row.  Slices of at most 32 k entries mark winners in per-slice bitmaps
+    # and write the output from every CTA; longer slices gather ordered lists
+    # on one CTA.  Both sides of that bound, with and without row statistics.
+    rng = np.random.default_rng(41 + k)
+    lens = [16385, 70001, 131072, 131073, 262144, 300001, 524288, 524289]
+    x = rng.standard_normal((len(lens), max(lens))).astype(np.float32)
+    if stats:
+        got = _gpu_topk_with_stats(x, k, lens)
+    else:
+        got = gpu_topk(x, k, row_len=lens)
+    assert np.array_equal(got, oracle.topk(x.astype(np.float64), lens, k))
+
+
+def test_topk_cluster_threshold_ties_across_slices():
+    # 1500 entries above and 200 entries exactly at the k-th value spread over
+    # every slice of the cluster: the ties are taken lowest index first
+    # across slices.
+    rng = np.random.default_rng(43)
+    n_rows, n = 6, 100000
+    x = rng.random((n_rows, n), dtype=np.float32)
+    for r in range(n_rows):
+        pos = rng.permutation(n)
+        x[r, pos[:1500]] = 5.0 + rng.random(1500, dtype=np.float32)
+        x[r, pos[1500:1700]] = 3.0
+    lens = [n - 3 * r for r in range(n_rows)]
+    ref = oracle.topk(x.astype(np.float64), lens, 2048)
+    assert np.array_equal(gpu_topk(x, 2048, row_len=lens), ref)
+    assert np.array_equal(_gpu_topk_with_stats(x, 2048, lens), ref)
+
+
 @pytest.mark.parametrize("n_tied", [300, 1000])
 def test_topk_exact_ties_at_the_threshold(n_tied):
     # 1500 entries above, n_tied entries exactly equal at the k-th value and
