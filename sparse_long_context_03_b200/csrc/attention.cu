@@ -343,25 +343,50 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) sparse_decode_split_kernel(
 }
 
 // Merge the split-K partials of one (sequence, head): one CTA of D threads.
+// The splits' running maxima are loaded in parallel and reduced; then each
+// thread folds the splits in order, eight at a time with their loads issued
+// together (the partials sit in L2, so a load-per-step chain would pay the
+// L2 latency once per split).
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const float *__restrict__ part, int Hq, int Hkv,
                                                            int nsplit, uint16_t *__restrict__ out,
                                                            float *__restrict__ lse) {
+    constexpr int kBatch = 8;
+    __shared__ float red[D / 32];
     const int bh = blockIdx.x;
     const int b = bh / Hq, h = bh % Hq;
     const int G = Hq / Hkv, g = h / G, hh = h % G;
     const float *p0 = part + ((size_t)(b * Hkv + g) * nsplit) * 8 * (D + 2) + (size_t)hh * (D + 2);
     const size_t stride = (size_t)8 * (D + 2);
+    const int d = threadIdx.x;
     float M = -INFINITY;
-    for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, p0[sp * stride + D]);
+    for (int sp = d; sp < nsplit; sp += D) M = fmaxf(M, p0[sp * stride + D]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+    if ((d & 31) == 0) red[d >> 5] = M;
+    __syncthreads();
+    M = red[0];
+#pragma unroll
+    for (int w = 1; w < D / 32; ++w) M = fmaxf(M, red[w]);
     const float Mref = M == -INFINITY ? 0.f : M;
     float L = 0.f, acc = 0.f;
-    const int d = threadIdx.x;
-    for (int sp = 0; sp < nsplit; ++sp) {
-        const float *p = p0 + sp * stride;
-        const float f = fast_exp2(p[D] - Mref);
-        L = fmaf(p[D + 1], f, L);
-        acc = fmaf(p[d], f, acc);
+    for (int sp0 = 0; sp0 < nsplit; sp0 += kBatch) {
+        float pv[kBatch], mv[kBatch], lv[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            const float *p = p0 + (size_t)min(sp0 + j, nsplit - 1) * stride;
+            pv[j] = p[d];
+            mv[j] = p[D];
+            lv[j] = p[D + 1];
+        }
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            if (sp0 + j < nsplit) {
+                const float f = fast_exp2(mv[j] - Mref);
+                L = fmaf(lv[j], f, L);
+                acc = fmaf(pv[j], f, acc);
+            }
+        }
     }
     out[(size_t)bh * D + d] = float_to_bf16_bits(L > 0.f ? acc / L : 0.f);
     if (lse != nullptr && d == 0) lse[bh] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
@@ -371,10 +396,16 @@ struct DecodeSplit {
     int chunk, nsplit;
 };
 
-// Enough splits to put ~16 warps on each of the 148 SMs, 16-key aligned.
-DecodeSplit decode_split(int B, int Hkv, int k) {
+// Upper bound on resident split warps that workspaces are sized for (148
+// SMs x 16 warps); a launch never uses more splits than this allows.
+constexpr int kSplitSlotsBound = 148 * 16;
+
+// Split the k index rows of each (sequence, group) pair so that all pairs'
+// warps are resident at once (`slots` = warps the device holds): one wave,
+// no tail of a few warps running alone.  Chunks are 16-key aligned.
+DecodeSplit decode_split(int B, int Hkv, int k, int slots) {
     const int pairs = B * Hkv > 0 ? B * Hkv : 1;
-    int want = (148 * 16 + pairs - 1) / pairs;
+    int want = slots / pairs;
     const int max_split = (k + kBlk - 1) / kBlk;
     want = want < 1 ? 1 : (want > max_split ? max_split : want);
     int chunk = (k + want - 1) / want;
@@ -391,6 +422,34 @@ bool dispatch_d(int D, F &&f) {
         default: return false;
     }
 }
+
+// Split warps the current device holds at once (SMs x resident one-warp
+// CTAs of the split kernel), looked up once per device, at most
+// kSplitSlotsBound.
+template <int D>
+int decode_split_slots() {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> cached[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return kSplitSlotsBound;
+    int v = cached[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
+        constexpr int smem = kWarpsPerCta * warp_smem_bytes<D>();
+        int sms = 0, per_sm = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            set_smem_at_least<sparse_decode_split_kernel<D>>(smem) == cudaSuccess &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_decode_split_kernel<D>,
+                                                          kWarpsPerCta * 32, smem) == cudaSuccess &&
+            sms > 0 && per_sm > 0)
+            v = sms * per_sm * kWarpsPerCta;
+        else
+            v = kSplitSlotsBound;
+        cached[dev].store(v, std::memory_order_relaxed);
+    }
+    return v < kSplitSlotsBound ? v : kSplitSlotsBound;
+}
+
+int decode_split_slots_for(int D) { return D == 64 ? decode_split_slots<64>() : decode_split_slots<128>(); }
 
 }  // namespace
 
@@ -425,7 +484,7 @@ cudaError_t launch_sparse_prefill(const uint16_t *Q, const uint16_t *K, const ui
 
 size_t decode_attention_workspace_bytes(int B, int Hq, int Hkv, int D, int k) {
     (void)Hq;
-    const DecodeSplit s = decode_split(B, Hkv, k);
+    const DecodeSplit s = decode_split(B, Hkv, k, kSplitSlotsBound);
     return (size_t)B * Hkv * s.nsplit * 8 * (D + 2) * sizeof(float);
 }
 
@@ -435,7 +494,8 @@ cudaError_t launch_sparse_decode(const uint16_t *q, const uint16_t *k_cache, con
                                  size_t ws_bytes, uint16_t *out, float *lse, cudaStream_t stream) {
     if (B == 0) return cudaSuccess;
     if (ws_bytes < decode_attention_workspace_bytes(B, Hq, Hkv, D, k)) return cudaErrorInvalidValue;
-    const DecodeSplit s = decode_split(B, Hkv, k);
+    if (D != 64 && D != 128) return cudaErrorInvalidValue;
+    const DecodeSplit s = decode_split(B, Hkv, k, decode_split_slots_for(D));
     const int items = B * Hkv * s.nsplit;
     const int grid = (items + kWarpsPerCta - 1) / kWarpsPerCta;
     float *part = static_cast<float *>(ws);
@@ -530,7 +590,8 @@ cudaError_t launch_sparse_decode_fixed_scratch(const uint16_t *q, const uint16_t
     float *part = fixed_scratch_on_current_device(&err);
     if (part == nullptr) return err;
     // Same split rule as the workspace variant, capped so the partials fit.
-    DecodeSplit s = decode_split(B, Hkv, k);
+    if (D != 64 && D != 128) return cudaErrorInvalidValue;
+    DecodeSplit s = decode_split(B, Hkv, k, decode_split_slots_for(D));
     if (s.nsplit > cap) {
         int chunk = (k + cap - 1) / cap;
         chunk = (chunk + kBlk - 1) / kBlk * kBlk;

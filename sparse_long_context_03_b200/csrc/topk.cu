@@ -630,6 +630,7 @@ struct ClusterExtra {
     uint32_t slice_cand[kClusterSize];
     uint32_t slice_chosen[kClusterSize];
     uint32_t ncand;
+    uint32_t wred[kWarps][kClusterSize];  // per-warp partial sums of slice_above
 };
 
 __host__ __device__ constexpr size_t cluster_smem_bytes(int k) { return smem_bytes(k) + sizeof(ClusterExtra); }
@@ -746,10 +747,23 @@ __global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads,
     }
     __syncthreads();
     cluster.sync();
-    for (int b = tid; b < kNB; b += kThreads) {
-        uint32_t sum = 0;
-        for (int q = 0; q < kClusterSize; ++q) sum += cluster.map_shared_rank(sm.hist, q)[b];
-        cx.ghist[b] = sum;
+    {
+        // thread j adds buckets 4j..4j+3 of every slice: one 16-byte remote
+        // load per slice (the remote load count, not its latency, is the cost)
+        static_assert(kNB == 4 * kThreads, "four buckets per thread");
+        uint4 s4 = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int q = 0; q < kClusterSize; ++q) {
+            const uint4 v = reinterpret_cast<const uint4 *>(cluster.map_shared_rank(sm.hist, q))[tid];
+            s4.x += v.x;
+            s4.y += v.y;
+            s4.z += v.z;
+            s4.w += v.w;
+        }
+        cx.ghist[4 * tid] = s4.x;
+        cx.ghist[4 * tid + 1] = s4.y;
+        cx.ghist[4 * tid + 2] = s4.z;
+        cx.ghist[4 * tid + 3] = s4.w;
     }
     __syncthreads();
     find_threshold_bin(cx.ghist, (uint32_t)k, sm.red, sm.bcast);
@@ -761,19 +775,37 @@ __global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads,
     const int bm_words = (chunk + 31) / 32;
     const bool usual = cnt <= (uint32_t)kSmallCand && bm_words <= k;
     if (usual) {
-        if (warp < kClusterSize) {  // warp q reads slice q's counts
-            const uint32_t *hq = cluster.map_shared_rank(sm.hist, warp);
-            uint32_t a = 0;
-            for (int b = (int)Bt + 1 + lane; b < kNB; b += 32) a += hq[b];
+        // every slice's entries above Bt: thread j sums its buckets 4j..4j+3
+        // above Bt in each slice (16-byte remote loads, only by threads that
+        // own such buckets), then the block reduces the eight sums
+        uint32_t a[kClusterSize];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
-            if (lane == 0) {
-                cx.slice_above[warp] = a;
-                cx.slice_cand[warp] = hq[Bt];
-                cx.slice_chosen[warp] = 0;
+        for (int q = 0; q < kClusterSize; ++q) a[q] = 0;
+        if (4 * tid + 3 > (int)Bt) {
+#pragma unroll
+            for (int q = 0; q < kClusterSize; ++q) {
+                const uint4 v = reinterpret_cast<const uint4 *>(cluster.map_shared_rank(sm.hist, q))[tid];
+                a[q] = (4 * tid > (int)Bt ? v.x : 0u) + (4 * tid + 1 > (int)Bt ? v.y : 0u) +
+                       (4 * tid + 2 > (int)Bt ? v.z : 0u) + v.w;
             }
         }
+#pragma unroll
+        for (int q = 0; q < kClusterSize; ++q) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) a[q] += __shfl_xor_sync(0xFFFFFFFFu, a[q], o);
+            if (lane == 0) cx.wred[warp][q] = a[q];
+        }
+        if (tid < kClusterSize) {
+            cx.slice_cand[tid] = cluster.map_shared_rank(sm.hist, tid)[Bt];
+            cx.slice_chosen[tid] = 0;
+        }
         if (tid == 0) cx.ncand = 0;
+        __syncthreads();
+        if (tid < kClusterSize) {
+            uint32_t t = 0;
+            for (int w = 0; w < kWarps; ++w) t += cx.wred[w][tid];
+            cx.slice_above[tid] = t;
+        }
         for (int w = tid; w < bm_words; w += kThreads) bm[w] = 0;
         __syncthreads();
     }
