@@ -620,20 +620,31 @@ __global__ void __launch_bounds__(kThreads) topk_rows_bitmap_kernel(const float 
 
 constexpr int kClusterSize = 8;
 
+constexpr int kCoarse = 64;             // super-buckets of the histogram exchange
+constexpr int kFine = kNB / kCoarse;     // buckets per super-bucket
+static_assert(kNB == 4 * kThreads && kFine == 32 && kCoarse * kClusterSize == kThreads, "exchange layout");
+
 struct ClusterExtra {
-    uint32_t ghist[kNB];   // the row's histogram (sum over the cluster)
     float range[2];        // this slice's min, max
     uint32_t counts[2];    // this slice's winners, candidates
+    uint32_t coarse[kCoarse];                 // this slice's super-bucket counts
+    uint32_t allc[kClusterSize][kCoarse];     // every slice's super-bucket counts
+    uint32_t allf[kClusterSize][kFine];       // every slice's buckets of the threshold super-bucket
+    uint32_t sel[8];                          // super-bucket, entries above it; Bt, need, n_above, cnt, Bt - 32 S
     // usual case: per slice, entries above the threshold bucket, entries in
     // it, and chosen candidates; this slice's candidates written so far
     uint32_t slice_above[kClusterSize];
     uint32_t slice_cand[kClusterSize];
     uint32_t slice_chosen[kClusterSize];
     uint32_t ncand;
-    uint32_t wred[kWarps][kClusterSize];  // per-warp partial sums of slice_above
 };
 
-__host__ __device__ constexpr size_t cluster_smem_bytes(int k) { return smem_bytes(k) + sizeof(ClusterExtra); }
+// Dynamic shared memory of the cluster kernel: the single-CTA layout, the
+// exchange area, then the largest bucket of each 16-entry group of the slice
+// (slices of at most 32 k entries: 2 k groups of 2 bytes).
+__host__ __device__ constexpr size_t cluster_smem_bytes(int k) {
+    return smem_bytes(k) + sizeof(ClusterExtra) + ((size_t)4 * k + 15) / 16 * 16;
+}
 
 __global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads, 2)
     topk_rows_cluster_kernel(const float *__restrict__ scores, int64_t ld, int row_begin,
@@ -662,6 +673,10 @@ __global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads,
     const int chunk = ((n + kClusterSize - 1) / kClusterSize + 15) / 16 * 16;
     const int lo = min(n, rank * chunk), m = min(n, lo + chunk) - lo;
     const float *srow = row + lo;
+    // start this slice's trip to L2 now: the range lookup below waits on a
+    // global load anyway, and the histogram pass then reads from L2
+    for (int i0 = tid * kVec; i0 < m; i0 += kChunk)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(srow + i0));
 
     // ---- value range of the row
     float vmin = INFINITY, vmax = -INFINITY;
@@ -737,83 +752,143 @@ __global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads,
     }
     const float scale = __fdiv_rn((float)kNB * 0.99999f, range);
 
-    // ---- histogram of this slice, then of the row
+    // ---- histogram of this slice, and the largest bucket of each 16-entry
+    // group (for the collect pass to skip groups below the threshold bucket)
+    uint32_t *bm = reinterpret_cast<uint32_t *>(alist);  // usual case: this slice's bitmap
+    uint16_t *gmax = reinterpret_cast<uint16_t *>(smem_raw + smem_bytes(k) + sizeof(ClusterExtra));
+    const int bm_words = (chunk + 31) / 32;
+    const bool small_slice = bm_words <= k;  // chunk <= 32 k: bitmap and group maxima fit
     for (int i0 = tid * kVec; i0 < m; i0 += kChunk) {
         float x[kVec];
         const int c = load_vals(srow, i0, m, x);
+        uint32_t gm = 0;
 #pragma unroll
         for (int j = 0; j < kVec; ++j)
-            if (j < c) atomicAdd(&sm.hist[bucket_of(x[j], vmin, scale)], 1u);
+            if (j < c) {
+                const uint32_t b = bucket_of(x[j], vmin, scale);
+                atomicAdd(&sm.hist[b], 1u);
+                gm = max(gm, b);
+            }
+        if (small_slice) gmax[i0 >> 4] = (uint16_t)gm;  // i0 is a multiple of kVec = 16
+    }
+    __syncthreads();
+    {
+        // super-bucket s = buckets 32 s .. 32 s + 31: eight threads' four buckets
+        const uint4 h = reinterpret_cast<const uint4 *>(sm.hist)[tid];
+        uint32_t v = h.x + h.y + h.z + h.w;
+        v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+        v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
+        v += __shfl_xor_sync(0xFFFFFFFFu, v, 4);
+        if ((tid & 7) == 0) cx.coarse[tid >> 3] = v;
     }
     __syncthreads();
     cluster.sync();
-    {
-        // thread j adds buckets 4j..4j+3 of every slice: one 16-byte remote
-        // load per slice (the remote load count, not its latency, is the cost)
-        static_assert(kNB == 4 * kThreads, "four buckets per thread");
-        uint4 s4 = make_uint4(0u, 0u, 0u, 0u);
+
+    // ---- the row's threshold bucket, in two small exchanges: every slice's
+    // super-bucket counts, then every slice's 32 buckets of the super-bucket
+    // that holds the k-th entry
+    cx.allc[tid / kCoarse][tid % kCoarse] = cluster.map_shared_rank(cx.coarse, tid / kCoarse)[tid % kCoarse];
+    __syncthreads();
+    if (warp == 0) {
+        // lane l holds super-buckets 2l and 2l + 1
+        uint32_t c0 = 0, c1 = 0;
 #pragma unroll
         for (int q = 0; q < kClusterSize; ++q) {
-            const uint4 v = reinterpret_cast<const uint4 *>(cluster.map_shared_rank(sm.hist, q))[tid];
-            s4.x += v.x;
-            s4.y += v.y;
-            s4.z += v.z;
-            s4.w += v.w;
+            c0 += cx.allc[q][2 * lane];
+            c1 += cx.allc[q][2 * lane + 1];
         }
-        cx.ghist[4 * tid] = s4.x;
-        cx.ghist[4 * tid + 1] = s4.y;
-        cx.ghist[4 * tid + 2] = s4.z;
-        cx.ghist[4 * tid + 3] = s4.w;
+        const uint32_t own = c0 + c1;
+        uint32_t v = own;  // becomes the sum over lanes >= this one
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, v, o);
+            if (lane + o < 32) v += y;
+        }
+        const uint32_t above = v - own, kk = (uint32_t)k;
+        if (above < kk && kk <= above + c1) {
+            cx.sel[0] = 2 * lane + 1;
+            cx.sel[1] = above;
+        } else if (above + c1 < kk && kk <= above + c1 + c0) {
+            cx.sel[0] = 2 * lane;
+            cx.sel[1] = above + c1;
+        }
     }
     __syncthreads();
-    find_threshold_bin(cx.ghist, (uint32_t)k, sm.red, sm.bcast);
-    const uint32_t Bt = sm.bcast[0];
-    const uint32_t need = sm.bcast[1];
-    const uint32_t n_above = sm.bcast[2];
-    const uint32_t cnt = cx.ghist[Bt];
-    uint32_t *bm = reinterpret_cast<uint32_t *>(alist);  // usual case: this slice's bitmap
-    const int bm_words = (chunk + 31) / 32;
-    const bool usual = cnt <= (uint32_t)kSmallCand && bm_words <= k;
+    const int S = (int)cx.sel[0];
+    if (tid < kClusterSize * kFine)
+        cx.allf[tid / kFine][tid % kFine] = cluster.map_shared_rank(sm.hist, tid / kFine)[S * kFine + tid % kFine];
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t f = 0;
+#pragma unroll
+        for (int q = 0; q < kClusterSize; ++q) f += cx.allf[q][lane];
+        uint32_t v = f;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, v, o);
+            if (lane + o < 32) v += y;
+        }
+        const uint32_t above = cx.sel[1] + (v - f), kk = (uint32_t)k;
+        if (above < kk && kk <= above + f) {
+            cx.sel[2] = (uint32_t)(S * kFine + lane);
+            cx.sel[3] = kk - above;
+            cx.sel[4] = above;
+            cx.sel[5] = f;
+            cx.sel[6] = (uint32_t)lane;
+        }
+    }
+    __syncthreads();
+    const uint32_t Bt = cx.sel[2];
+    const uint32_t need = cx.sel[3];
+    const uint32_t n_above = cx.sel[4];
+    const uint32_t cnt = cx.sel[5];
+    const int jt = (int)cx.sel[6];
+    const int n_groups = (m + kVec - 1) / kVec;
+    // usual case (the same decision on every CTA: it depends on the row, not
+    // the slice): up to kSmallCand candidates, then the list of groups to
+    // revisit in the rest of the candidate arrays
+    const bool usual = cnt <= (uint32_t)kSmallCand && small_slice && chunk / kVec <= kCap - kSmallCand;
     if (usual) {
-        // every slice's entries above Bt: thread j sums its buckets 4j..4j+3
-        // above Bt in each slice (16-byte remote loads, only by threads that
-        // own such buckets), then the block reduces the eight sums
-        uint32_t a[kClusterSize];
-#pragma unroll
-        for (int q = 0; q < kClusterSize; ++q) a[q] = 0;
-        if (4 * tid + 3 > (int)Bt) {
-#pragma unroll
-            for (int q = 0; q < kClusterSize; ++q) {
-                const uint4 v = reinterpret_cast<const uint4 *>(cluster.map_shared_rank(sm.hist, q))[tid];
-                a[q] = (4 * tid > (int)Bt ? v.x : 0u) + (4 * tid + 1 > (int)Bt ? v.y : 0u) +
-                       (4 * tid + 2 > (int)Bt ? v.z : 0u) + v.w;
-            }
-        }
-#pragma unroll
-        for (int q = 0; q < kClusterSize; ++q) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a[q] += __shfl_xor_sync(0xFFFFFFFFu, a[q], o);
-            if (lane == 0) cx.wred[warp][q] = a[q];
-        }
+        // every slice's counts follow from the two exchanges
         if (tid < kClusterSize) {
-            cx.slice_cand[tid] = cluster.map_shared_rank(sm.hist, tid)[Bt];
+            uint32_t a = 0;
+            for (int sb = S + 1; sb < kCoarse; ++sb) a += cx.allc[tid][sb];
+            for (int j = jt + 1; j < kFine; ++j) a += cx.allf[tid][j];
+            cx.slice_above[tid] = a;
+            cx.slice_cand[tid] = cx.allf[tid][jt];
             cx.slice_chosen[tid] = 0;
         }
         if (tid == 0) cx.ncand = 0;
-        __syncthreads();
-        if (tid < kClusterSize) {
-            uint32_t t = 0;
-            for (int w = 0; w < kWarps; ++w) t += cx.wred[w][tid];
-            cx.slice_above[tid] = t;
-        }
         for (int w = tid; w < bm_words; w += kThreads) bm[w] = 0;
         __syncthreads();
+        // No cluster barrier here: no CTA leaves before the barrier after the
+        // collect, the histograms read above are not written again, and the
+        // candidate lists written by other CTAs are not read before it.
+    } else {
+        cluster.sync();  // every remote read of the histograms is done (the paths below may leave early)
     }
-    cluster.sync();  // every remote read of the histograms is done
     if (usual) {
         uint32_t coff = 0;  // this slice's first slot in the row's candidate list
         for (int q = 0; q < rank; ++q) coff += cx.slice_cand[q];
-        for (int i0 = tid * kVec; i0 < m; i0 += kChunk) {
+        // the groups holding an entry at or above the threshold bucket (about
+        // one in five), listed so that the loads below are one round for the
+        // whole CTA instead of one per group a thread owns
+        uint32_t *glist = sm.ckey + kSmallCand;
+        if (tid == 0) cx.counts[0] = 0;
+        __syncthreads();
+        for (int g0 = 0; g0 < n_groups; g0 += kThreads) {
+            const int g = g0 + tid;
+            const bool hit = g < n_groups && gmax[g] >= Bt;
+            const unsigned bal = __ballot_sync(0xFFFFFFFFu, hit);
+            uint32_t base = 0;
+            if (lane == 0 && bal) base = atomicAdd(&cx.counts[0], (uint32_t)__popc(bal));
+            base = __shfl_sync(0xFFFFFFFFu, base, 0);
+            if (hit) glist[base + __popc(bal & ((1u << lane) - 1u))] = (uint32_t)g;
+        }
+        __syncthreads();
+        const int n_hit = (int)cx.counts[0];
+        for (int gi = tid; gi < n_hit; gi += kThreads) {
+            const int i0 = (int)glist[gi] * kVec;
             float x[kVec];
             const int c = load_vals(srow, i0, m, x);
             uint32_t win = 0;
