@@ -802,11 +802,29 @@ def omega_union(plan, L, k, width=16, fracs=(0.125, 0.25, 0.5, 0.75, 0.99), samp
 def run_profile_case(args):
     """One GPU, no timing: `fused` runs the fused indexer + top-k of the
     workload twice, `attention` selects once and runs the prefill attention
-    twice (the second launch of each is the one to capture); `omega-union`
-    prints the union of Omega over 16 adjacent queries as JSON."""
+    twice, `decode-indexer` runs the decode indexer of a decode workload
+    twice with only its FP8 key cache on the device (the second launch of
+    each is the one to capture); `omega-union` prints the union of Omega
+    over 16 adjacent queries as JSON."""
     from sparse_long_context_03_b200 import build, dsa, inputs
     build.build()
     cfg = inputs.config(args.config)
+    if args.profile_case == "decode-indexer":
+        if cfg.B <= 0:
+            raise SystemExit("--profile-case decode-indexer needs a decode workload (--config 3)")
+        g = inputs.decode_inputs(cfg, device="cuda", B=args.decode_batch)
+        for key in ("k_cache", "v_cache", "q"):
+            del g[key]
+        torch.cuda.empty_cache()
+        B, L = g["q8"].shape[0], g["max_seq_len"]
+        scores = torch.empty(B, (L + 3) // 4 * 4, dtype=torch.float32, device="cuda")
+        for _ in range(2):
+            dsa.decode_indexer_scores(g["q8"], g["sq"], g["w"], g["k8_cache"], g["sk_cache"], g["block_table"],
+                                      g["seq_lens"], L, scores)
+        torch.cuda.synchronize()
+        print(json.dumps({"workload": cfg.name, "profile_case": "decode-indexer", "B": B,
+                          "device_bytes": torch.cuda.memory_allocated(), "status": "ok"}))
+        return 0
     d = inputs.prefill_inputs(cfg, device="cuda")
     plan = dsa.PrefillPlan(cfg.L, cfg.HI, cfg.dI, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, chunk_rows=args.chunk_rows,
                            device="cuda", fused=False if args.unfused else True)
@@ -843,7 +861,7 @@ def main():
                     help="materialise the score matrix per chunk and run dsa_topk (instead of dsa_indexer_topk)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="sequences in the decode workload (default: the decode-b32 layer's 32)")
-    ap.add_argument("--profile-case", default=None, choices=["fused", "attention", "omega-union"],
+    ap.add_argument("--profile-case", default=None, choices=["fused", "attention", "omega-union", "decode-indexer"],
                     help="run one untimed case on one GPU for a profiler capture (no bench line)")
     args = ap.parse_args()
 
