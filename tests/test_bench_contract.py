@@ -68,3 +68,36 @@ def test_oracle_sample_rows_and_extrapolation():
     tiny = inputs.config(0, L=9)
     tok_s, full = bench.extrapolate_tok_per_s(tiny, [4], 2.0)  # mean of t+1 over t<9 is 5
     assert full == pytest.approx(2.0 * 9) and tok_s == pytest.approx(9 / 18.0)
+
+
+def test_omega_union_counts_distinct_selected_keys():
+    # 16 adjacent query rows; row t selects {t, t+1, ..., t+k-1} clipped to
+    # -1 padding past 40: the union of rows t0..t0+15 is t0..min(39, t0+15+k-1)
+    import torch
+
+    k, L = 4, 64
+
+    class Plan:
+        pass
+
+    plan = Plan()
+    idx = torch.full((L, k), -1, dtype=torch.int32)
+    for t in range(L):
+        for j in range(k):
+            if t + j < 40:
+                idx[t, j] = t + j
+    plan.idx = idx
+    res = bench.omega_union(plan, L, k, width=16, fracs=(0.0, 0.5), samples=1)
+    first = res["t~0"]  # rows 0..15: keys 0..18
+    assert first["mean_union"] == 19 and first["min"] == 19 and first["max"] == 19
+    assert abs(first["of_width_k"] - 19 / 64) < 1e-12
+    second = res["t~32"]  # rows 32..47: keys 32..39 only
+    assert second["mean_union"] == 8
+
+
+def test_profile_case_choices_are_accepted():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--help"], capture_output=True, text=True,
+                         cwd=ROOT, timeout=300)
+    assert out.returncode == 0
+    for case in ("fused", "attention", "omega-union", "decode-indexer"):
+        assert case in out.stdout
