@@ -207,6 +207,25 @@ def test_topk_cluster_threshold_ties_across_slices():
     assert np.array_equal(_gpu_topk_with_stats(x, 2048, lens), ref)
 
 
+@pytest.mark.parametrize("n_tied", [300, 7000])
+def test_topk_cluster_crowded_threshold_bucket(n_tied):
+    # Few long rows (one cluster each) whose threshold bucket holds more
+    # than 256 entries: 300 exact ties take the gathered ordered lists, 7000
+    # (more than fit in shared memory) the whole-row radix select; both with
+    # and without row statistics.
+    rng = np.random.default_rng(44 + n_tied)
+    n_rows, n = 4, 120000
+    x = rng.random((n_rows, n), dtype=np.float32)
+    for r in range(n_rows):
+        pos = rng.permutation(n)
+        x[r, pos[:1500]] = 5.0 + rng.random(1500, dtype=np.float32)
+        x[r, pos[1500:1500 + n_tied]] = 3.0
+    lens = [n - 5 * r for r in range(n_rows)]
+    ref = oracle.topk(x.astype(np.float64), lens, 2048)
+    assert np.array_equal(gpu_topk(x, 2048, row_len=lens), ref)
+    assert np.array_equal(_gpu_topk_with_stats(x, 2048, lens), ref)
+
+
 @pytest.mark.parametrize("n_tied", [300, 1000])
 def test_topk_exact_ties_at_the_threshold(n_tied):
     # 1500 entries above, n_tied entries exactly equal at the k-th value and
