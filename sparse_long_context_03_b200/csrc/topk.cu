@@ -639,18 +639,32 @@ struct ClusterExtra {
     uint32_t ncand;
 };
 
-// Dynamic shared memory of the cluster kernel: the single-CTA layout, the
-// exchange area, then the largest bucket of each 16-entry group of the slice
-// (slices of at most 32 k entries: 2 k groups of 2 bytes).
-__host__ __device__ constexpr size_t cluster_smem_bytes(int k) {
-    return smem_bytes(k) + sizeof(ClusterExtra) + ((size_t)4 * k + 15) / 16 * 16;
+// Dynamic shared memory of the cluster kernel: the single-CTA layout and the
+// exchange area, then (cluster_gmax_groups) the largest bucket of each
+// 16-entry group of the slice, 2 bytes per group.
+__host__ __device__ constexpr size_t cluster_base_bytes(int k) {
+    return (smem_bytes(k) + sizeof(ClusterExtra) + 15) / 16 * 16;
+}
+constexpr size_t kClusterSmemMax = 220 * 1024;
+
+// Groups the group-maxima array holds for rows of at most max_len entries:
+// enough for a slice of the usual case (at most 32 k entries) when it fits
+// next to the rest; rows whose slices need more take the gathered-list path.
+int cluster_gmax_groups(int k, int max_len) {
+    const long long chunk_max = ((long long)(max_len + kClusterSize - 1) / kClusterSize + 15) / 16 * 16;
+    long long want = chunk_max / kVec;
+    if (want > 2ll * k) want = 2ll * k;
+    want = (want + 7) / 8 * 8;  // whole 16-byte units
+    const long long room = ((long long)kClusterSmemMax - (long long)cluster_base_bytes(k)) / 2;
+    if (want > room) want = room / 8 * 8;
+    return want > 0 ? (int)want : 0;
 }
 
 __global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads, 2)
     topk_rows_cluster_kernel(const float *__restrict__ scores, int64_t ld, int row_begin,
                              const int32_t *__restrict__ row_len, int max_len, int k, int32_t *__restrict__ idx,
                              const float *__restrict__ row_stats, const uint32_t *__restrict__ row_keyrange,
-                             int n_rows) {
+                             int n_rows, int gmax_groups) {
     namespace cgs = cooperative_groups;
     cgs::cluster_group cluster = cgs::this_cluster();
     const int rank = (int)cluster.block_rank();
@@ -755,9 +769,10 @@ __global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kThreads,
     // ---- histogram of this slice, and the largest bucket of each 16-entry
     // group (for the collect pass to skip groups below the threshold bucket)
     uint32_t *bm = reinterpret_cast<uint32_t *>(alist);  // usual case: this slice's bitmap
-    uint16_t *gmax = reinterpret_cast<uint16_t *>(smem_raw + smem_bytes(k) + sizeof(ClusterExtra));
+    uint16_t *gmax = reinterpret_cast<uint16_t *>(smem_raw + cluster_base_bytes(k));
     const int bm_words = (chunk + 31) / 32;
-    const bool small_slice = bm_words <= k;  // chunk <= 32 k: bitmap and group maxima fit
+    // chunk <= 32 k and chunk / 16 groups fit: bitmap and group maxima fit
+    const bool small_slice = bm_words <= k && chunk / kVec <= gmax_groups;
     for (int i0 = tid * kVec; i0 < m; i0 += kChunk) {
         float x[kVec];
         const int c = load_vals(srow, i0, m, x);
@@ -1026,12 +1041,13 @@ cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_ro
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (max_len >= 16384 && n_rows < (sms > 0 ? sms : 148)) {
         // few long rows: a cluster of CTAs per row keeps every SM busy
-        const size_t csmem = cluster_smem_bytes(k);
-        if (csmem > 220 * 1024) return cudaErrorInvalidValue;
+        const int gmax_groups = cluster_gmax_groups(k, max_len);
+        const size_t csmem = cluster_base_bytes(k) + (size_t)gmax_groups * 2;
+        if (csmem > kClusterSmemMax) return cudaErrorInvalidValue;
         cudaError_t e = set_smem_at_least<topk_rows_cluster_kernel>(csmem);
         if (e != cudaSuccess) return e;
         topk_rows_cluster_kernel<<<n_rows * kClusterSize, kThreads, csmem, stream>>>(
-            scores, ld, row_begin, row_len, max_len, k, idx, row_stats, row_keyrange, n_rows);
+            scores, ld, row_begin, row_len, max_len, k, idx, row_stats, row_keyrange, n_rows, gmax_groups);
         return cudaGetLastError();
     }
     if (bitmap_smem_bytes(max_len) <= (size_t)kBitmapSmemMax) {
@@ -1051,6 +1067,6 @@ cudaError_t launch_topk(const float *scores, int64_t ld, int row_begin, int n_ro
     return cudaGetLastError();
 }
 
-bool topk_k_supported(int k) { return cluster_smem_bytes(k) <= 220 * 1024; }
+bool topk_k_supported(int k) { return cluster_base_bytes(k) <= kClusterSmemMax; }
 
 }  // namespace dsa

@@ -207,6 +207,18 @@ def test_topk_cluster_threshold_ties_across_slices():
     assert np.array_equal(_gpu_topk_with_stats(x, 2048, lens), ref)
 
 
+@pytest.mark.parametrize("k", [30000, 40000])
+def test_topk_cluster_large_k(k):
+    # k up to the ABI's bound on the per-row cluster path (few rows, long
+    # row bound): random rows past k, one below it
+    rng = np.random.default_rng(k)
+    lens = [150000, 90001, k - 1]
+    x = rng.standard_normal((len(lens), max(lens))).astype(np.float32)
+    ref = oracle.topk(x.astype(np.float64), lens, k)
+    assert np.array_equal(gpu_topk(x, k, row_len=lens), ref)
+    assert np.array_equal(_gpu_topk_with_stats(x, k, lens), ref)
+
+
 @pytest.mark.parametrize("n_tied", [300, 7000])
 def test_topk_cluster_crowded_threshold_bucket(n_tied):
     # Few long rows (one cluster each) whose threshold bucket holds more
