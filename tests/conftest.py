@@ -12,7 +12,7 @@ GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
-    config.addinivalue_line("markers", "slow: full-size workload, minutes on the GPU box")
+    config.addinivalue_line("markers", "slow: full-size workload, minutes on one GPU")
 
 
 def read_golden(name):
