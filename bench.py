@@ -809,20 +809,30 @@ def run_profile_case(args):
     from sparse_long_context_03_b200 import build, dsa, inputs
     build.build()
     cfg = inputs.config(args.config)
-    if args.profile_case == "decode-indexer":
+    if args.profile_case in ("decode-indexer", "decode-topk"):
         if cfg.B <= 0:
-            raise SystemExit("--profile-case decode-indexer needs a decode workload (--config 3)")
+            raise SystemExit(f"--profile-case {args.profile_case} needs a decode workload (--config 3)")
         g = inputs.decode_inputs(cfg, device="cuda", B=args.decode_batch)
         for key in ("k_cache", "v_cache", "q"):
             del g[key]
         torch.cuda.empty_cache()
         B, L = g["q8"].shape[0], g["max_seq_len"]
         scores = torch.empty(B, (L + 3) // 4 * 4, dtype=torch.float32, device="cuda")
-        for _ in range(2):
+        for _ in range(2 if args.profile_case == "decode-indexer" else 1):
             dsa.decode_indexer_scores(g["q8"], g["sq"], g["w"], g["k8_cache"], g["sk_cache"], g["block_table"],
                                       g["seq_lens"], L, scores)
+        if args.profile_case == "decode-topk":
+            # the top-k of the decode rows with each row's range given (the
+            # same path as the decode chain, where the indexer records it)
+            valid = torch.arange(scores.shape[1], device="cuda")[None, :] < g["seq_lens"][:, None].long()
+            lo = torch.where(valid, scores, torch.full_like(scores, float("inf"))).amin(1)
+            hi = torch.where(valid, scores, torch.full_like(scores, float("-inf"))).amax(1)
+            stats = torch.stack([lo, hi], 1).repeat(1, 4).contiguous()
+            idx = torch.empty(B, cfg.k, dtype=torch.int32, device="cuda")
+            for _ in range(2):
+                dsa.topk(scores, 0, B, cfg.k, idx, row_len=g["seq_lens"], max_len=L, row_stats=stats)
         torch.cuda.synchronize()
-        print(json.dumps({"workload": cfg.name, "profile_case": "decode-indexer", "B": B,
+        print(json.dumps({"workload": cfg.name, "profile_case": args.profile_case, "B": B,
                           "device_bytes": torch.cuda.memory_allocated(), "status": "ok"}))
         return 0
     d = inputs.prefill_inputs(cfg, device="cuda")
@@ -861,7 +871,8 @@ def main():
                     help="materialise the score matrix per chunk and run dsa_topk (instead of dsa_indexer_topk)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="sequences in the decode workload (default: the decode-b32 layer's 32)")
-    ap.add_argument("--profile-case", default=None, choices=["fused", "attention", "omega-union", "decode-indexer"],
+    ap.add_argument("--profile-case", default=None, choices=["fused", "attention", "omega-union", "decode-indexer",
+                                                               "decode-topk"],
                     help="run one untimed case on one GPU for a profiler capture (no bench line)")
     args = ap.parse_args()
 

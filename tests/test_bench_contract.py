@@ -99,5 +99,5 @@ def test_profile_case_choices_are_accepted():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--help"], capture_output=True, text=True,
                          cwd=ROOT, timeout=300)
     assert out.returncode == 0
-    for case in ("fused", "attention", "omega-union", "decode-indexer"):
+    for case in ("fused", "attention", "omega-union", "decode-indexer", "decode-topk"):
         assert case in out.stdout
