@@ -114,6 +114,38 @@ def measure_read_peaks(dsa):
                    f"HBM: one pass over 4 GiB, best of 5; CUDA events"}
 
 
+def _avg_back_to_back_ms(fn, n=20):
+    """Mean time of one fn() call over n back-to-back calls between two CUDA
+    events (after three warm-up calls): the GPU never waits for the host, so
+    the figure is the kernels' time.  For buffers well beyond L2, a pass does
+    not find the previous pass's data in L2: the previous pass's tail is
+    evicted before this pass reaches it."""
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        fn()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        fn()
+    b.record(stream)
+    b.synchronize()
+    return a.elapsed_time(b) / n
+
+
+def measure_single_pass_read(dsa, n_bytes):
+    """Read bandwidth of one pass over a buffer of n_bytes (beyond L2) with
+    the library's read probe, averaged over back-to-back passes: what a
+    kernel that reads that many bytes once can reach, ramp-up and tail
+    included."""
+    sink = torch.zeros(4, dtype=torch.int32, device="cuda")
+    buf = torch.ones((n_bytes + 15) // 16 * 4, dtype=torch.int32, device="cuda")
+    ms = _avg_back_to_back_ms(lambda: dsa.read_probe(buf, 1, sink))
+    gbs = buf.numel() * 4 / (ms / 1e3) / 1e9
+    del buf
+    return gbs
+
+
 # ----------------------------------------------------------------------------
 # distributed plumbing
 # ----------------------------------------------------------------------------
@@ -832,8 +864,20 @@ def run_profile_case(args):
             for _ in range(2):
                 dsa.topk(scores, 0, B, cfg.k, idx, row_len=g["seq_lens"], max_len=L, row_stats=stats)
         torch.cuda.synchronize()
-        print(json.dumps({"workload": cfg.name, "profile_case": args.profile_case, "B": B,
-                          "device_bytes": torch.cuda.memory_allocated(), "status": "ok"}))
+        line = {"workload": cfg.name, "profile_case": args.profile_case, "B": B,
+                "device_bytes": torch.cuda.memory_allocated(), "status": "ok"}
+        if args.profile_case == "decode-indexer":
+            # the indexer reads the key cache and its scales once: what one
+            # read pass over that many bytes reaches, and the indexer's time
+            n_bytes = g["k8_cache"].numel() + g["sk_cache"].numel() * 4
+            line["single_pass_read_gbs"] = measure_single_pass_read(dsa, n_bytes)
+            line["cache_bytes"] = n_bytes
+            ms = _avg_back_to_back_ms(lambda: dsa.decode_indexer_scores(g["q8"], g["sq"], g["w"], g["k8_cache"],
+                                                                        g["sk_cache"], g["block_table"],
+                                                                        g["seq_lens"], L, scores))
+            line["indexer_us"] = ms * 1e3
+            line["indexer_gbs"] = n_bytes / (ms / 1e3) / 1e9
+        print(json.dumps(line))
         return 0
     d = inputs.prefill_inputs(cfg, device="cuda")
     plan = dsa.PrefillPlan(cfg.L, cfg.HI, cfg.dI, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, chunk_rows=args.chunk_rows,
@@ -942,6 +986,14 @@ def main():
                                "unit": "GB/s", "frac": byts / (us / 1e6) / 1e9 / pk["hbm_gbs"],
                                "algorithmic_bytes": byts},
                   "gpu_launches_per_step": 4, "clocks": dclk}
+        if rank == 0:
+            # a step this short cannot reach the multi-GB copy figure: beside
+            # it, one read pass over the step's own bytes, measured here
+            sp = measure_single_pass_read(_dsa, byts)
+            decode["roofline"].update({
+                "single_pass_read_gbs": sp, "frac_of_single_pass": byts / (us / 1e6) / 1e9 / sp,
+                "single_pass_note": "dsa_read_probe, one pass over a buffer of the step's algorithmic bytes, "
+                                    "mean of 20 back-to-back passes"})
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             decode_host = decode_host_inputs(db)
         del db
