@@ -480,9 +480,11 @@ __global__ void __maxnreg__(EpiShape<HI>::kMaxRegs) indexer_tc_kernel(const __gr
 //              (sequence, step, length, page validity) and copies each
 //              sequence's query rows, in sequence order, into one of two
 //              swizzled query slots;
-//   MMA        (SP/2) x (dI/32) UMMAs per step into an (SP/2) x N column
-//              accumulator.  Its fixed cost per step (barrier waits, fences,
-//              commits: several hundred cycles) is what sizes the step;
+//   MMA        two warps take alternate steps, (SP/2) x (dI/32) UMMAs per
+//              step into an (SP/2) x N column accumulator.  One thread's
+//              cost per step (barrier waits, fences, eight UMMAs and two
+//              commits: about 0.7 us) was most of the step period with one
+//              MMA warp; two overlap it;
 //   epilogue   kDecGroups groups of four warps take alternate steps: per tile
 //              each thread owns one key, reads its N columns, ReLU and the
 //              head-weighted sum, the two scales, and stores one score.
@@ -495,9 +497,9 @@ constexpr int kDecPage = 64;       // tokens per cache page
 constexpr int kDecGroups = 2;
 constexpr int kDecProducers = 4;
 constexpr int kDecProducer0 = 4 * kDecGroups;         // warps 0 .. 4G-1: epilogue
-constexpr int kDecMmaWarp = kDecProducer0 + kDecProducers;
-constexpr int kDecThreads = (kDecMmaWarp + 1) * 32;
-// 13 warps leave four on one scheduler, whose 16K registers cap a thread at 128.
+constexpr int kDecMmaWarp = kDecProducer0 + kDecProducers;  // two MMA warps: kDecMmaWarp, kDecMmaWarp + 1
+constexpr int kDecThreads = (kDecMmaWarp + 2) * 32;
+// 14 warps leave four on one scheduler, whose 16K registers cap a thread at 128.
 constexpr int kDecMaxRegs = 128;
 
 template <int N, int DI>
@@ -605,13 +607,13 @@ __global__ void __maxnreg__(kDecMaxRegs) indexer_decode_tc_kernel(
         }
         for (int q = 0; q < 2; ++q) {
             tc::mbar_init(qfull_bar(q), 1);
-            tc::mbar_init(qempty_bar(q), 1);
+            tc::mbar_init(qempty_bar(q), 2);  // one release per MMA warp
         }
         for (int a = 0; a < A; ++a) {
             tc::mbar_init(tfull_bar(a), 1);
             tc::mbar_init(tempty_bar(a), 4);
         }
-        tc::mbar_init(mma_done_bar, 1);
+        tc::mbar_init(mma_done_bar, 2);
         tc::fence_mbar_init();
     }
     if (warp == kDecMmaWarp) {
@@ -745,36 +747,52 @@ __global__ void __maxnreg__(kDecMaxRegs) indexer_decode_tc_kernel(
                 (void)tc::mbar_wait(full_bar(li % S), (uint32_t)((li / S) & 1), lim);
         }
         __syncwarp();
-    } else if (warp == kDecMmaWarp) {
+    } else if (warp >= kDecMmaWarp) {
         // ------------------------------------------------------------ UMMA
+        // Two MMA warps take alternate steps: one thread's issue cost per
+        // step (eight small UMMAs, two commits, the waits) is most of a step
+        // period, and two threads overlap it.  Accumulator a = li % A serves
+        // one warp only (A even).  Both warps walk every step of the range,
+        // find its sequence from the step prefix, and release each query
+        // slot when they pass its sequence (the release counts two arrivals),
+        // so a warp that had no step of a short sequence still releases its
+        // slot; a warp waits for a slot's query only when it uses it.  No
+        // barrier runs two phases ahead of a wait: refilling a stage, an
+        // accumulator or a slot needs this warp's own earlier release.
+        static_assert(Lay::kAccBufs % 2 == 0, "an accumulator serves one MMA warp");
+        const int mw = warp - kDecMmaWarp;
         if (lane == 0) {
             bool ok = true;
-            int cur_b = -1, qc = -1;
+            int cur_b = -1, qc = -1, b = 0;
+            bool have_q = false;
             for (int li = 0; li < nsteps; ++li) {
-                const int s = li % S, a = li % A;
-                if (!tc::mbar_wait_sleep(full_bar(s), (li / S) & 1, kWaitLimitNs, kIssuerSleepNs)) {
-                    ok = false;
-                    break;
-                }
-                const volatile int *mp = reinterpret_cast<volatile int *>(smem + s * Lay::kStageBytes + Lay::kMeta);
-                const int4 meta = make_int4(mp[0], mp[1], mp[2], mp[3]);
-                if (meta.x != cur_b) {
+                const int gi = i0 + li;
+                while (prefix[b + 1] <= gi) ++b;  // prefix[B] = total > gi
+                if (b != cur_b) {
                     if (qc >= 0) tc::umma_commit(qempty_bar(qc & 1));
-                    cur_b = meta.x;
+                    cur_b = b;
                     ++qc;
+                    have_q = false;
+                }
+                if ((li & 1) != mw) continue;
+                const int s = li % S, a = li % A;
+                if (!have_q) {
                     if (!tc::mbar_wait_sleep(qfull_bar(qc & 1), (qc >> 1) & 1, kWaitLimitNs, kIssuerSleepNs)) {
                         ok = false;
                         break;
                     }
+                    have_q = true;
                 }
-                if (!tc::mbar_wait_sleep(tempty_bar(a), ((li / A) & 1) ^ 1, kWaitLimitNs, kIssuerSleepNs)) {
+                if (!tc::mbar_wait_sleep(full_bar(s), (li / S) & 1, kWaitLimitNs, kIssuerSleepNs) ||
+                    !tc::mbar_wait_sleep(tempty_bar(a), ((li / A) & 1) ^ 1, kWaitLimitNs, kIssuerSleepNs)) {
                     ok = false;
                     break;
                 }
                 tc::tc_fence_after();
                 const uint32_t kaddr = sbase + s * Lay::kStageBytes;
                 const uint32_t qaddr = sbase + Lay::kQ + (qc & 1) * Lay::kQBytes;
-                const int pages = min(SP, (meta.z + kDecPage - 1) / kDecPage - SP * meta.y);
+                const int st = gi - prefix[b];
+                const int pages = min(SP, (seq_len_of(b) + kDecPage - 1) / kDecPage - SP * st);
 #pragma unroll
                 for (int t = 0; t < T; ++t) {
                     if (2 * t >= pages) break;
@@ -788,6 +806,7 @@ __global__ void __maxnreg__(kDecMaxRegs) indexer_decode_tc_kernel(
                 tc::umma_commit(tfull_bar(a));
             }
             if (!ok) record_timeout();
+            // every UMMA either warp issued has completed before TMEM is freed
             tc::umma_commit(mma_done_bar);
             (void)tc::mbar_wait(mma_done_bar, 0, kWaitLimitNs);
         }
